@@ -1,0 +1,284 @@
+"""Pins for the float64 oracle: each check comes from somewhere other than the oracle itself.
+
+Sources of truth used here: hand-derived worked examples (tests/golden/hand_examples.json),
+the SVD polar factor (LAPACK), the spectral characterisation of the iteration (singular
+vectors kept, singular values mapped by the scalar polynomial), textbook special cases and
+a brute-force triple-loop matmul.  The last test plants mistakes in a copy of the
+iteration and checks that these pins catch every one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")))
+
+
+def rel(a, b):
+    return np.linalg.norm(np.asarray(a) - np.asarray(b)) / max(np.linalg.norm(np.asarray(b)), 1e-300)
+
+
+def orthogonal(rng, n):
+    q, r = np.linalg.qr(rng.standard_normal((n, n)))
+    return q * np.sign(np.diag(r))
+
+
+def with_singular_values(rng, rows, cols, s):
+    k = min(rows, cols)
+    P = orthogonal(rng, rows)[:, :k]
+    Q = orthogonal(rng, cols)[:, :k]
+    return (P * s) @ Q.T
+
+
+# ---------------------------------------------------------------- primitive
+
+def test_matmul_primitive_matches_triple_loop():
+    rng = np.random.default_rng(1)
+    A = rng.standard_normal((8, 12))
+    B = rng.standard_normal((12, 8))
+    C = np.zeros((8, 8))
+    for i in range(8):
+        for j in range(8):
+            s = 0.0
+            for k in range(12):
+                s += A[i, k] * B[k, j]
+            C[i, j] = s
+    assert np.max(np.abs(C - A @ B)) < 1e-13
+
+
+def test_gram_step_matches_triple_loop():
+    # The Gram and B X products of one step, written as loops over a 4x6 matrix.
+    rng = np.random.default_rng(2)
+    X = rng.standard_normal((4, 6))
+    a, b, c = O.QUINTIC
+    A = [[sum(X[i, k] * X[j, k] for k in range(6)) for j in range(4)] for i in range(4)]
+    AA = [[sum(A[i][k] * A[k][j] for k in range(4)) for j in range(4)] for i in range(4)]
+    Bm = [[b * A[i][j] + c * AA[i][j] for j in range(4)] for i in range(4)]
+    Xn = [[a * X[i, j] + sum(Bm[i][k] * X[k, j] for k in range(4)) for j in range(6)] for i in range(4)]
+    assert rel(O.ns_iteration(X, a, b, c), np.array(Xn)) < 1e-14
+
+
+# ---------------------------------------------------------------- worked examples
+
+def test_momentum_worked_example():
+    g = GOLD["momentum"]
+    M1 = O.momentum_lerp(np.array([[g["M"]]]), np.array([[g["G"]]]), g["beta"])
+    assert abs(M1[0, 0] - g["M1"]) < 1e-15
+    U = O.nesterov_blend(np.array([[g["G"]]]), M1, g["beta"], True)
+    assert abs(U[0, 0] - g["U_nesterov"]) < 1e-15
+    U = O.nesterov_blend(np.array([[g["G"]]]), M1, g["beta"], False)
+    assert abs(U[0, 0] - g["U_plain"]) < 1e-15
+
+
+def test_frobenius_worked_example():
+    g = GOLD["frobenius"]
+    assert O.frobenius_norm(np.array(g["X"])) == g["norm"]
+    assert np.allclose(O.frobenius_normalize(np.array(g["X"]), 0.0), g["normalized"], atol=1e-15)
+
+
+@pytest.mark.parametrize("key,abc,k", [("cubic_k1", O.CUBIC, 1), ("cubic_k2", O.CUBIC, 2), ("quintic_k1", O.QUINTIC, 1)])
+def test_ns_diagonal_worked_example(key, abc, k):
+    g = GOLD["ns_diagonal"]
+    out = O.newton_schulz(np.array(g["U"]), k, abc, g["eps"])
+    assert np.max(np.abs(out - np.array(g[key]))) < 1e-14
+
+
+def test_ns_tall_worked_example():
+    g = GOLD["ns_tall"]
+    out = O.newton_schulz(np.array(g["U"]), 1, O.CUBIC, g["eps"])
+    assert out.shape == (3, 2)
+    assert np.max(np.abs(out - np.array(g["cubic_k1"]))) < 1e-14
+
+
+def test_parameter_write_worked_example():
+    g = GOLD["write"]
+    assert abs(O.shape_scale(3, 2) - g["scale"]) < 1e-15
+    W1 = O.parameter_write(np.array(g["W"]), np.array(g["O"]), g["lr"], g["weight_decay"])
+    assert np.max(np.abs(W1 - np.array(g["W1"]))) < 1e-10
+
+
+def test_muon_step_worked_example():
+    # W = 0, M = 0, G = diag(3, 4)/c: U is a positive multiple of diag(3, 4), so with eps = 0
+    # the orthogonalised direction is the cubic_k1 diagonal, whatever beta is.
+    g = GOLD["ns_diagonal"]
+    G = np.array(g["U"]) / 7.0
+    hp = O.Hyper(lr=0.5, beta=0.9, weight_decay=0.0, eps=0.0, nesterov=True, ns_steps=1, abc=O.CUBIC)
+    W1, M1, Oo = O.muon_step(np.zeros((2, 2)), G, np.zeros((2, 2)), hp)
+    assert np.max(np.abs(M1 - 0.1 * G)) < 1e-16
+    assert np.max(np.abs(Oo - np.array(g["cubic_k1"]))) < 1e-14
+    assert np.max(np.abs(W1 + 0.5 * np.array(g["cubic_k1"]))) < 1e-14
+
+
+def test_quintic_constants():
+    g = GOLD["quintic_constants"]
+    assert abs(O.scalar_map(1.0, 1) - g["phi_at_1"]) < 1e-12
+    xs = np.linspace(0.0, 1.0, 200001)
+    ys = O.scalar_map(xs, 1)
+    assert abs(xs[np.argmax(ys)] - g["argmax_on_unit_interval"]) < 1e-4
+    assert abs(ys.max() - g["max_on_unit_interval"]) < 1e-5
+
+
+# ---------------------------------------------------------------- special cases
+
+def test_momentum_special_cases():
+    rng = np.random.default_rng(3)
+    G, M = rng.standard_normal((5, 7)), rng.standard_normal((5, 7))
+    # beta = 0: no memory, the direction is the gradient
+    M1 = O.momentum_lerp(M, G, 0.0)
+    assert np.array_equal(M1, G)
+    assert np.array_equal(O.nesterov_blend(G, M1, 0.0, True), G)
+    # beta = 1: the buffer never moves
+    M1 = O.momentum_lerp(M, G, 1.0)
+    assert np.array_equal(M1, M)
+    assert np.array_equal(O.nesterov_blend(G, M1, 1.0, True), M)
+    # G = M: a fixed point of the lerp, and of the blend
+    M1 = O.momentum_lerp(M, M, 0.95)
+    assert np.max(np.abs(M1 - M)) < 1e-15
+    assert np.max(np.abs(O.nesterov_blend(M, M1, 0.95, True) - M)) < 1e-15
+
+
+def test_norm_against_lapack():
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((33, 17))
+    assert abs(O.frobenius_norm(X) - np.linalg.norm(X, "fro")) < 1e-12
+    assert abs(O.frobenius_norm(X) - math.sqrt(np.sum(np.linalg.svd(X, compute_uv=False) ** 2))) < 1e-12
+
+
+def test_shape_scale():
+    assert O.shape_scale(1536, 1536) == 1.0
+    assert O.shape_scale(1536, 6144) == 1.0
+    assert abs(O.shape_scale(6144, 1536) - 2.0) < 1e-15
+    assert abs(O.shape_scale(3072, 1024) - math.sqrt(3.0)) < 1e-15
+    assert abs(O.shape_scale(12288, 3072) - 2.0) < 1e-15
+
+
+# ---------------------------------------------------------------- iteration vs plain definitions
+
+@pytest.mark.parametrize("shape", [(32, 48), (48, 32), (40, 40)])
+def test_cubic_converges_to_polar_factor(shape):
+    rng = np.random.default_rng(5)
+    s = np.linspace(0.1, 1.0, min(shape))
+    X = with_singular_values(rng, *shape, s)
+    out = O.newton_schulz(X, 40, O.CUBIC, 0.0)
+    assert rel(out, O.polar_factor(X)) < 1e-12
+
+
+def test_cubic_polar_on_gaussian_256():
+    # The 256x256 N(0,1) matrix from seed 0: sigma_min / ||X||_F is small, so the step count
+    # is chosen from it: log(0.5/s_min)/log(1.5) steps to reach the quadratic basin, plus 8.
+    X = np.random.default_rng(0).standard_normal((256, 256))
+    s = np.linalg.svd(X, compute_uv=False)
+    smin = s[-1] / math.sqrt(np.sum(s * s))
+    k = math.ceil(math.log(0.5 / smin) / math.log(1.5)) + 8
+    out = O.newton_schulz(X, k, O.CUBIC, 0.0)
+    assert rel(out, O.polar_factor(X)) < 1e-10, k
+
+
+@pytest.mark.parametrize("shape", [(24, 40), (40, 24), (30, 30)])
+@pytest.mark.parametrize("k", [1, 2, 5])
+@pytest.mark.parametrize("abc", [O.QUINTIC, O.CUBIC, (2.0, -1.5, 0.5)])
+def test_iteration_equals_spectral_map(shape, k, abc):
+    rng = np.random.default_rng(6)
+    X = rng.standard_normal(shape)
+    out = O.newton_schulz(X, k, abc, 1e-7)
+    assert rel(out, O.spectral_newton_schulz(X, k, abc, 1e-7)) < 1e-12
+
+
+def test_spectral_map_ill_conditioned():
+    # singular values spanning 1e-6 .. 1, as in the conditioning stress set
+    rng = np.random.default_rng(7)
+    s = np.exp(rng.uniform(np.log(1e-6), 0.0, 48))
+    X = with_singular_values(rng, 48, 96, s)
+    for k in (5, 10):
+        assert rel(O.newton_schulz(X, k), O.spectral_newton_schulz(X, k)) < 1e-11
+
+
+# ---------------------------------------------------------------- invariants
+
+def test_invariants():
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((20, 36))
+    base = O.newton_schulz(X, 5)
+    # transpose symmetry: the tall path is the wide path transposed, exactly
+    assert np.array_equal(O.newton_schulz(X.T, 5), base.T)
+    # odd polynomial
+    assert np.array_equal(O.newton_schulz(-X, 5), -base)
+    # scale invariance (exact with eps = 0, up to rounding)
+    b0 = O.newton_schulz(X, 5, eps=0.0)
+    assert rel(O.newton_schulz(123.0 * X, 5, eps=0.0), b0) < 1e-13
+    # orthogonal equivariance
+    P, Q = orthogonal(rng, 20), orthogonal(rng, 36)
+    assert rel(O.newton_schulz(P @ X @ Q, 5), P @ base @ Q) < 1e-12
+
+
+def test_orthonormal_rows_fixed_points():
+    rng = np.random.default_rng(9)
+    Q = orthogonal(rng, 40)[:16, :]  # 16x40, orthonormal rows
+    # the bare cubic step keeps Q where it is
+    assert np.max(np.abs(O.ns_iteration(Q, *O.CUBIC) - Q)) < 1e-14
+    # with normalisation the result is a scalar multiple of Q: phi^k(1/(sqrt(r)+eps)) Q
+    eps = 1e-7
+    for abc in (O.CUBIC, O.QUINTIC):
+        for k in (1, 5, 30):
+            scale = O.scalar_map(1.0 / (math.sqrt(16) + eps), k, abc)
+            assert rel(O.newton_schulz(Q, k, abc, eps), scale * Q) < 1e-13
+    # for the cubic the scalar goes to 1
+    assert abs(O.scalar_map(1.0 / (4 + eps), 40, O.CUBIC) - 1.0) < 1e-12
+
+
+def test_zero_input_stays_finite():
+    # eps keeps the normalisation finite; the zero matrix maps to zero
+    out = O.newton_schulz(np.zeros((8, 16)), 5)
+    assert np.array_equal(out, np.zeros((8, 16)))
+
+
+def test_ns_flops_counts():
+    # square: 3 m^3 + m^3 per step; wide m x n: 3 m^2 n + m^3
+    assert O.ns_flops(1536, 1536, 1) == 4 * 1536 ** 3
+    assert O.ns_flops(6144, 1536, 5) == 5 * (3 * 1536 * 1536 * 6144 + 1536 ** 3)
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def _mutants():
+    a, b, c = O.QUINTIC
+
+    def drop_c(X):
+        A = X @ X.T
+        return a * X + (b * A) @ X
+
+    def wrong_gram(X):
+        # the Gram of the other side, still multiplied from the left (square inputs only)
+        A = X.T @ X
+        B = b * A + c * (A @ A)
+        return a * X + B @ X
+
+    def wrong_sign(X):
+        A = X @ X.T
+        B = b * A - c * (A @ A)
+        return a * X + B @ X
+
+    def transposed_update(X):
+        A = X @ X.T
+        B = b * A + c * (A @ A)
+        return a * X + (B @ X) @ np.eye(X.shape[1])[::-1]
+
+    return [drop_c, wrong_gram, wrong_sign, transposed_update]
+
+
+@pytest.mark.parametrize("mutant", _mutants(), ids=lambda f: f.__name__)
+def test_pins_catch_planted_mistakes(mutant, monkeypatch):
+    """Each plausible slip in the iteration must fail the spectral pin."""
+    import oracle.muon_oracle as mo
+
+    rng = np.random.default_rng(10)
+    X = rng.standard_normal((30, 30))
+    good = mo.newton_schulz(X, 3)
+    monkeypatch.setattr(mo, "ns_iteration", lambda Y, a, b, c: mutant(Y))
+    bad = mo.newton_schulz(X, 3)
+    assert rel(good, O.spectral_newton_schulz(X, 3)) < 1e-12
+    assert rel(bad, O.spectral_newton_schulz(X, 3)) > 1e-3
