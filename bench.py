@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Benchmark of the Muon optimizer step on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload d24] [--impl muon|reference]
+
+A step is one muon_step over the whole parameter set (momentum + norm, k
+Newton-Schulz iterations of Gram / polynomial / update, parameter write), with
+W, G and M resident in HBM.  Inputs are synthetic and seeded
+(muon_newton_schulz_07_b200.inputs).  Under torchrun every rank steps its own
+parameter set (weak scaling) and the time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Muon optimizer steps/s per param set; NS TFLOP/s & % of B200 bf16 dense peak"
+UNIT = "steps/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["muon", "reference"], default="muon")
+    ap.add_argument("--workload", default="d24", choices=["gpt2s", "d24", "l38b", "stress"])
+    ap.add_argument("--ns-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-budget-s", type=float, default=150.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS if k in p}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops_by_kind(shapes, k):
+    """Algorithmic flops per step (2 per multiply-add; the symmetric products counted once)."""
+    gram = poly = upd = 0
+    for r, c in shapes:
+        m, n = min(r, c), max(r, c)
+        gram += m * m * n
+        poly += m ** 3
+        upd += 2 * m * m * n
+    return {"gram": k * gram, "poly": k * poly, "update": k * upd}
+
+
+def bytes_by_kind(shapes, elem=2):
+    n = sum(r * c for r, c in shapes)
+    # momentum_norm: read G, M; write M1 and X0.  write: read W and the final X, write W.
+    return {"momentum_norm": 4 * elem * n, "write": 3 * elem * n}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = [d for d in threadpool_info() if d.get("user_api") == "blas"]
+        if info:
+            return int(max(d.get("num_threads", 1) for d in info))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="muon_clocks_", suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+
+        sm = [num(r[1]) for r in rows]
+        mx = [num(r[2]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(num(r[3]) for r in rows)}
+
+
+def gpu_index_for(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ---------------------------------------------------------------- oracle timings (CPU)
+
+def oracle_sample(wl, max_seconds=30.0):
+    """Time the float64 oracle on one matrix of each distinct shape; extrapolate to the set."""
+    import numpy as np
+
+    import oracle as O
+    from muon_newton_schulz_07_b200 import inputs as I
+
+    first = {}
+    for i, s in enumerate(wl.shapes):
+        first.setdefault(s, i)
+    counts = {s: wl.shapes.count(s) for s in first}
+    hp = O.Hyper(lr=0.02, beta=0.95, weight_decay=0.0, eps=1e-7, nesterov=True, ns_steps=5)
+    per_shape = {}
+    t_all = time.perf_counter()
+    for s, i in first.items():
+        W, G, M = I.weight(wl, i).astype(np.float64), I.gradient(wl, 1, i).astype(np.float64), \
+            I.momentum(wl, i).astype(np.float64)
+        t0 = time.perf_counter()
+        O.muon_step(W, G, M, hp)
+        per_shape[s] = time.perf_counter() - t0
+        if time.perf_counter() - t_all > max_seconds:
+            break
+    if len(per_shape) < len(first):
+        # budget ran out: scale the rest by flops from the timed shapes
+        rate = sum(O.ns_flops(*s, 5) for s in per_shape) / sum(per_shape.values())
+        for s in first:
+            per_shape.setdefault(s, O.ns_flops(*s, 5) / rate)
+    step_s = sum(counts[s] * per_shape[s] for s in first)
+    sample = "one matrix of each distinct shape (" + ", ".join(f"{r}x{c}" for r, c in first) + \
+        f"), float64 NumPy oracle, scaled by shape counts to the {len(wl.shapes)}-matrix set (extrapolated)"
+    return step_s, sample
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    from muon_newton_schulz_07_b200 import inputs as I
+
+    import numpy as np
+
+    import oracle as O
+
+    wl = I.WORKLOADS[args.workload]
+    first = {}
+    for i, s in enumerate(wl.shapes):
+        first.setdefault(s, i)
+    shapes = list(first)
+    counts = {s: wl.shapes.count(s) for s in shapes}
+    hp = O.Hyper(ns_steps=args.ns_steps)
+    times = {s: [] for s in shapes}
+    t_begin = time.perf_counter()
+    done = 0
+    for it in range(args.warmup + args.steps):
+        s = shapes[it % len(shapes)]
+        i = first[s]
+        W, G, M = (I.weight(wl, i).astype(np.float64), I.gradient(wl, 1 + it, i).astype(np.float64),
+                   I.momentum(wl, i).astype(np.float64))
+        t0 = time.perf_counter()
+        O.muon_step(W, G, M, hp)
+        dt = time.perf_counter() - t0
+        if it >= args.warmup:
+            times[s].append(dt)
+            done += 1
+        if time.perf_counter() - t_begin > args.reference_budget_s and all(times[x] for x in shapes):
+            break
+    step_s = sum(counts[s] * statistics.median(times[s]) for s in shapes)
+    value = 1.0 / step_s
+    cores = blas_threads()
+    sample = (f"each timed step is one matrix of one distinct shape, cycling through "
+              f"{', '.join(f'{r}x{c}' for r, c in shapes)}; the full-set step time is the sum over shapes of "
+              f"count x median time (extrapolated)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": done,
+        "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "matrices": len(wl.shapes), "params": I.param_count(wl),
+                   "ns_steps": args.ns_steps},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- the Muon arm
+
+def run_muon(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    from muon_newton_schulz_07_b200 import binding as B
+    from muon_newton_schulz_07_b200 import inputs as I
+    from muon_newton_schulz_07_b200.optimizer import MuonStep
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = I.WORKLOADS[args.workload]
+    shapes = list(wl.shapes)
+    n = len(shapes)
+    k = args.ns_steps
+    dt = torch.bfloat16
+
+    def to_dev(a):
+        return torch.from_numpy(a).to(dev).to(dt)
+
+    # Every rank steps its own parameter set; gradients differ by rank through the step seed.
+    from concurrent.futures import ThreadPoolExecutor
+
+    def gen(fn):
+        with ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
+            return [to_dev(a) for a in ex.map(fn, range(n))]
+
+    W = gen(lambda i: I.weight(wl, i))
+    M = gen(lambda i: I.momentum(wl, i))
+    G_sets = [gen(lambda i, s=s: I.gradient(wl, 1 + s + 1000 * rank, i)) for s in range(2)]
+    op = MuonStep(shapes, dtype=dt, device=dev)
+    launches = op.launches_per_step(k)
+    stream = torch.cuda.current_stream(dev)
+
+    def sync_all():
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for i in range(args.warmup):
+        op(W, G_sets[i % 2], M, ns_steps=k)
+    sync_all()
+    if op.status() != B.MUON_OK:
+        raise RuntimeError("device status after warm-up is not OK")
+
+    clocks = ClockSampler(gpu_index_for(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    B.muon_profile_begin(op.handle, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync_all()
+    e0.record(stream)
+    for i in range(args.steps):
+        op(W, G_sets[i % 2], M, ns_steps=k)
+    e1.record(stream)
+    sync_all()
+    clk = clocks.stop()
+    ms_total = e0.elapsed_time(e1)
+    prof = B.muon_profile_end(op.handle)
+    status = op.status()
+    if status != B.MUON_OK:
+        raise RuntimeError(f"device status after the timed steps: {B.STATUS.get(status, status)}")
+    ms_per_step = max_over_ranks(ms_total / args.steps)
+    value = world * 1000.0 / ms_per_step
+
+    # ------------------------------------------------------------ end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        G_host = [[g.cpu().pin_memory() for g in gs] for gs in G_sets]
+        G_dev = [torch.empty_like(g) for g in G_sets[0]]
+        ksteps = max(1, min(args.steps, 20))
+        norms_host = torch.empty((ksteps, n), dtype=torch.float32).pin_memory()
+        h2d = sum(g.numel() * g.element_size() for g in G_host[0])
+        sync_all()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(ksteps):
+            for d, h in zip(G_dev, G_host[i % 2]):
+                d.copy_(h, non_blocking=True)
+            op(W, G_dev, M, ns_steps=k)
+            op.norms(out=norms_host[i])
+        f1.record(stream)
+        sync_all()
+        assert np.isfinite(norms_host.numpy()).all()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / ksteps)
+        e2e = {"value": world * 1000.0 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": 4 * n, "ms_per_step": e2e_ms, "steps": ksteps,
+               "path": "pinned host G -> device copy, MuonStep.__call__ (C ABI muon_step), norms -> pinned host"}
+
+    # ------------------------------------------------------------ roofline
+    peaks, peak_src = load_peaks()
+    fl = flops_by_kind(shapes, k)
+    by = bytes_by_kind(shapes)
+    kern = {kname: {"ms_total": ms, "launches": cnt, "ms_per_launch": (ms / cnt if cnt else None)}
+            for kname, (ms, cnt) in prof.items() if cnt}
+    dominant = max(kern, key=lambda x: kern[x]["ms_total"])
+    per_launch_units = {
+        "gram": fl["gram"] / k, "poly": fl["poly"] / k, "update": fl["update"] / k,
+        "momentum_norm": by["momentum_norm"], "write": by["write"],
+    }
+    if dominant in ("gram", "poly", "update"):
+        ach = per_launch_units[dominant] / (kern[dominant]["ms_per_launch"] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                "traffic": None, "kernel": f"ns_gemm_tc_kernel ({dominant})",
+                "peak_source": f"{peak_src} bf16_tflops_sustained"}
+    else:
+        ach = per_launch_units[dominant] / (kern[dominant]["ms_per_launch"] * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "traffic": None, "kernel": dominant, "peak_source": f"{peak_src} hbm_gbs"}
+    ns_ms = sum(kern[x]["ms_total"] for x in ("gram", "poly", "update") if x in kern) / args.steps
+    ns_flops = sum(fl.values())
+    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms > 0 else None
+    for kname, kd in kern.items():
+        if kname in ("gram", "poly", "update"):
+            kd["tflops"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e12
+            kd["frac_of_sustained_peak"] = kd["tflops"] / peaks["bf16_tflops_sustained"]
+        elif kname in ("momentum_norm", "write"):
+            kd["gbs"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e9
+            kd["frac_of_hbm"] = kd["gbs"] / peaks["hbm_gbs"]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        step_s, sample = oracle_sample(wl)
+        cpu = {"value": 1.0 / step_s, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "matrices": n, "params": I.param_count(wl), "ns_steps": k,
+                       "groups": op.n_groups, "parallelism": f"replica x{world} (one parameter set per GPU)",
+                       "l2": "inputs larger than L2 (W, G, M: %.2f GB per GPU), no flush" %
+                             (3 * 2 * I.param_count(wl) / 1e9),
+                       "description": wl.description},
+            "roofline": roof,
+            "ns": {"tflops": ns_tflops, "frac_of_sustained_peak": (ns_tflops / peaks["bf16_tflops_sustained"])
+                   if ns_tflops else None, "frac_of_burst_peak": (ns_tflops / peaks["bf16_tflops"])
+                   if ns_tflops else None, "ms_per_step": ns_ms, "flops_per_step": ns_flops},
+            "kernels": kern,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    op.close()
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        try:
+            run_muon(args, rank, world, local_rank)
+        finally:
+            dist.destroy_process_group()
+    else:
+        run_muon(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

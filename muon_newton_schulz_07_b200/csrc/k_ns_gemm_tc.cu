@@ -1,0 +1,323 @@
+// The Newton-Schulz products on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// One persistent kernel runs one stage of one Newton-Schulz iteration for every
+// matrix of the parameter set (all shape groups in one launch):
+//   Gram    A = s * X X^T          (s = 1/(||U||+eps)^2 on the first iteration)
+//   Poly    B = b * A + c * A A    (A symmetric, so A A = A A^T)
+//   Update  X' = s * (a * X + B X) (s = 1/(||U||+eps) on the first iteration)
+// which together are one step of the Newton-Schulz orthogonalisation the pages
+// name for Muon's matrix parameters (aiproducthub "开发者千美元训3.8B模型 击败GPT-2",
+// 影响 paragraph).
+//
+// Gram and Poly outputs are symmetric: only 256 x 256 macro tiles on or above
+// the diagonal are computed (two 128-row CTA tiles each); every element on or
+// above the diagonal is stored at (r, c) and mirrored to (c, r), so the result
+// is exactly symmetric.
+//
+// CTA layout (192 threads, one CTA per SM, persistent over a static
+// round-robin tile list):
+//   warp 0      TMA producer: 64 x 64 bf16 boxes, 128-byte swizzle, into a
+//               4-stage ring of {A 128 x 64, B 256 x 64} shared-memory tiles
+//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f16,
+//               M = 128, N = 256, K = 16, fp32 accumulators in TMEM, two
+//               accumulator buffers (2 x 256 columns) so the epilogue of one
+//               tile overlaps the main loop of the next
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, the fp32 combination
+//               with the auxiliary input (A for Poly, X for Update), bf16 cast,
+//               global stores (plus the mirrored store for Gram/Poly)
+// Operand B of Update is X itself in its row-major layout, i.e. MN-major; the
+// other operands are K-major.  All waits are bounded (see muon_device.cuh).
+#include <cuda_bf16.h>
+
+#include "muon_device.cuh"
+#include "muon_internal.h"
+
+namespace muon {
+namespace {
+
+constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK, STAGES = kTcStages;
+constexpr uint32_t BOX_BYTES = 64 * 64 * 2;             // one TMA box
+constexpr uint32_t A_STAGE = BM * BK * 2;               // 16 KB
+constexpr uint32_t B_STAGE = BN * BK * 2;               // 32 KB
+constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE;     // 48 KB
+constexpr uint32_t TMEM_COLS = 512;                     // 2 accumulators x 256 fp32 columns
+constexpr uint32_t BAR_BYTES = 256;
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+
+struct Tile {
+  int g, mat, row0, col0;
+};
+
+__device__ __forceinline__ Tile decode_tile(const TcParams& p, int t) {
+  int g = 0;
+  while (g + 1 < p.ngroups && p.g[g + 1].tile_begin <= t) ++g;
+  const TcGroup& G = p.g[g];
+  const int local = t - G.tile_begin;
+  const int mat = local / G.tiles_per_mat;
+  const int r = local - mat * G.tiles_per_mat;
+  Tile ti;
+  ti.g = g;
+  ti.mat = mat;
+  if (p.kind == kUpdate) {
+    const int tm = r / G.tdim;
+    ti.row0 = tm * BM;
+    ti.col0 = (r - tm * G.tdim) * BN;
+  } else {
+    // upper-triangle macro tile q = (I, J), I <= J, row-major; two row halves each
+    int q = r >> 1, I = 0;
+    while (q >= G.tdim - I) {
+      q -= G.tdim - I;
+      ++I;
+    }
+    ti.row0 = I * 256 + (r & 1) * BM;
+    ti.col0 = (I + q) * 256;
+  }
+  return ti;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& q, float* v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float* v) {
+  uint4 q;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  return q;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) ns_gemm_tc_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf_bar(a), 1);
+      mbar_init(acce_bar(a), 4);  // one arrival per epilogue warp
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int g = 0; g < p.ngroups; ++g) {
+      tma_prefetch_desc(&p.g[g].tm_a);
+      tma_prefetch_desc(&p.g[g].tm_b);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint64_t tmo = p.timeout_ns;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+        const Tile ti = decode_tile(p, t);
+        const TcGroup& G = p.g[ti.g];
+        bool ok = true;
+        for (int kb = 0; kb < G.kblocks; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full_bar(stage);
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + A_STAGE;
+          const int k0 = kb * BK;
+          tma_load_3d(sa, &G.tm_a, fb, k0, ti.row0, ti.mat);
+          tma_load_3d(sa + BOX_BYTES, &G.tm_a, fb, k0, ti.row0 + 64, ti.mat);
+          if (p.kind != kUpdate) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) tma_load_3d(sb + h * BOX_BYTES, &G.tm_b, fb, k0, ti.col0 + 64 * h, ti.mat);
+          } else {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) tma_load_3d(sb + h * BOX_BYTES, &G.tm_b, fb, ti.col0 + 64 * h, k0, ti.mat);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      // Do not leave the CTA while loads are still landing in shared memory:
+      // wait (bounded) until every stage's last armed phase has completed.
+      for (int i = 0; i < STAGES; ++i) {
+        if (*abort_flag) break;
+        (void)mbar_wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, p.status);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, p.kind == kUpdate ? 1 : 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+        const Tile ti = decode_tile(p, t);
+        const TcGroup& G = p.g[ti.g];
+        if (!mbar_wait_bounded(acce_bar(acc), acc_phase ^ 1u, tmo, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < G.kblocks; ++kb) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, tmo, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + A_STAGE;
+#pragma unroll
+          for (int j = 0; j < BK / 16; ++j) {
+            const uint64_t adesc = smem_desc_sw128(sa + 32u * j, 16, 1024);
+            const uint64_t bdesc = (p.kind == kUpdate) ? smem_desc_sw128(sb + 2048u * j, 8192, 1024)
+                                                       : smem_desc_sw128(sb + 32u * j, 16, 1024);
+            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | j) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty_bar(stage));  // frees the stage once these MMAs have read it
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(accf_bar(acc));  // accumulator ready for the epilogue
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const int row_in_tile = quad * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+      const Tile ti = decode_tile(p, t);
+      const TcGroup& G = p.g[ti.g];
+      if (!mbar_wait_bounded(accf_bar(acc), acc_phase, tmo, abort_flag, p.status)) break;
+      tc_fence_after();
+      float s = 1.0f;
+      if (p.use_scal) {
+        const float al = p.scal[2 * (G.scal_base + ti.mat) + 1];
+        s = (p.kind == kGram) ? al * al : al;
+      }
+      const int ld = G.out_ld;
+      const size_t mat_off = static_cast<size_t>(ti.mat) * G.mp * ld;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(G.out) + mat_off;
+      const __nv_bfloat16* aux = G.aux ? static_cast<const __nv_bfloat16*>(G.aux) + mat_off : nullptr;
+      const int gr = ti.row0 + row_in_tile;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        float v[32];
+        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the divergent stores below
+        tmem_ld_32cols(taddr + ch * 32, v);
+        if (ch == BN / 32 - 1) {
+          // all of this accumulator has been read: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acce_bar(acc));
+        }
+        const int gc0 = ti.col0 + ch * 32;
+        const bool symmetric = (p.kind != kUpdate);
+        if (symmetric && gc0 + 31 < gr) continue;  // strictly below the diagonal: mirrored from elsewhere
+        if (aux != nullptr) {
+          const uint4* ap = reinterpret_cast<const uint4*>(aux + static_cast<size_t>(gr) * ld + gc0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float a8[8];
+            unpack8(__ldg(ap + q), a8);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[8 * q + i] = s * fmaf(p.c_acc, v[8 * q + i], p.c_aux * a8[i]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = s * p.c_acc * v[i];
+        }
+        __nv_bfloat16* orow = out + static_cast<size_t>(gr) * ld + gc0;
+        if (!symmetric || gc0 >= gr) {
+          uint4* op = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) op[q] = pack8(v + 8 * q);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (gc0 + i >= gr) orow[i] = __float2bfloat16_rn(v[i]);
+        }
+        if (symmetric) {
+          // mirrored store: lanes hold consecutive rows, so each column store is coalesced
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (gc0 + i > gr) out[static_cast<size_t>(gc0 + i) * ld + gr] = __float2bfloat16_rn(v[i]);
+        }
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+size_t tc_smem_bytes() { return SMEM_BYTES; }
+
+cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s) {
+  if (p.total_tiles <= 0) return cudaSuccess;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
+  ns_gemm_tc_kernel<<<grid, kTcThreads, SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

@@ -1,0 +1,140 @@
+// Internal launch interfaces between the C ABI (muon_api.cu) and the kernels.
+// Nothing here is exported from libmuon.so.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+
+namespace muon {
+
+// Device status codes (written to the workspace status word; match muon_status_t).
+constexpr unsigned int kDevTimeout = 5;
+constexpr unsigned int kDevFault = 6;
+
+// Every workspace buffer is padded to multiples of this many rows/columns.
+constexpr int kPad = 256;
+
+// ------------------------------------------------------------------ elementwise
+// Elementwise kernels work on X-coordinate tiles of 64 x 128 (X is the oriented
+// matrix, min(rows,cols) x max(rows,cols), padded to multiples of kPad).
+constexpr int kEwTileR = 64;
+constexpr int kEwTileC = 128;
+constexpr int kEwThreads = 256;
+constexpr int kEwCluster = 8;       // CTAs per cluster in the momentum/norm kernel
+constexpr int kEwMatsPerLaunch = 192;
+
+enum Dtype : int { kBF16 = 0, kF32 = 1 };
+
+struct EwMat {
+  const void* src;   // G (step) or X (orthogonalize), rows x cols, caller's layout
+  void* mom;         // M, updated in place; nullptr: no momentum (U = src)
+  void* x;           // workspace X buffer of this matrix, mp x np, row stride np
+  int rows, cols;    // caller's shape
+  int mp, np;        // padded oriented shape
+  int trans;         // rows > cols: X = U^T
+  int tile_begin;    // first CTA (cluster aligned) of this matrix in the launch
+  int tiles_c;       // X tiles along np
+  int ntiles;        // X tiles of the padded matrix (mp/64 * np/128)
+  int scal_idx;      // slot of this matrix in the scalar / counter tables
+  int caller_idx;    // position in the caller's matrix list
+  int part_begin;    // first per-cluster partial slot
+  int nclusters;     // clusters covering this matrix
+};
+
+struct EwParams {
+  EwMat mat[kEwMatsPerLaunch];
+  int nmat;
+  int total_ctas;
+  float beta;
+  float eps;
+  int nesterov;
+  int vec_ok;              // every row of every matrix starts 16-byte aligned
+  float* partials;         // per-cluster sums of squares
+  float* scal;             // per matrix: {||U||_F, 1/(||U||_F + eps)}
+  unsigned int* counters;  // per matrix arrival counters, zero before the launch
+  float* norms;            // ||U||_F per matrix, caller order
+};
+
+struct WrMat {
+  void* w;           // W (updated in place) or O (written)
+  const void* x;     // final X of this matrix, mp x np, row stride np
+  int rows, cols, mp, np, trans;
+  int tile_begin;    // first CTA of this matrix
+  int tiles_c;       // tiles along the real n
+  int scal_idx;
+  float shape_scale; // sqrt(max(1, rows/cols))
+};
+
+struct WrParams {
+  WrMat mat[kEwMatsPerLaunch];
+  int nmat;
+  int total_ctas;
+  float lr, wd;
+  int store_only;   // 1: O = X (orthogonalize); 0: W = (1 - lr*wd) W - lr*s*X
+  int use_alpha;    // 1: X still unnormalised (k = 0), multiply by 1/(||U||+eps)
+  int vec_ok;
+  const float* scal;
+};
+
+cudaError_t launch_momentum_norm(const EwParams& p, Dtype io, Dtype xt, cudaStream_t s);
+cudaError_t launch_param_write(const WrParams& p, Dtype io, Dtype xt, cudaStream_t s);
+
+// ------------------------------------------------------------------ tcgen05 GEMMs
+constexpr int kTcBM = 128;
+constexpr int kTcBN = 256;
+constexpr int kTcBK = 64;
+constexpr int kTcStages = 4;
+constexpr int kTcMaxGroups = 6;
+constexpr int kTcThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+
+enum TcKind : int { kGram = 0, kPoly = 1, kUpdate = 2 };
+
+struct alignas(64) TcGroup {
+  CUtensorMap tm_a;     // operand A source (box 64 x 64 x 1, 128B swizzle)
+  CUtensorMap tm_b;     // operand B source
+  void* out;            // [cnt][rows][ld] bf16
+  const void* aux;      // [cnt][rows][ld] bf16 epilogue input, or nullptr
+  int cnt, mp, np;
+  int tiles_per_mat;
+  int tile_begin;
+  int kblocks;
+  int scal_base;
+  int tdim;             // Gram/Poly: mp/256 (triangle side); Update: np/256
+  int out_ld;
+  int pad_[3];
+};
+
+struct TcParams {
+  TcGroup g[kTcMaxGroups];
+  int ngroups;
+  int total_tiles;
+  int kind;
+  int use_scal;          // first iteration: fold the normalisation in
+  float c_acc, c_aux;    // out = s * (c_acc * acc + c_aux * aux)
+  const float* scal;
+  unsigned int* status;
+  unsigned long long timeout_ns;
+};
+
+size_t tc_smem_bytes();
+cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s);
+
+// ------------------------------------------------------------------ fp32 reference GEMMs
+struct SgParams {
+  const float* a; const float* b; float* c; const float* aux;
+  int M, N, K;
+  int lda, ldb, ldc;
+  long long sa, sb, sc;   // batch strides (elements)
+  int cnt;
+  int b_trans;            // 1: second operand is b^T (b row-major N x K)
+  float c_acc, c_aux;
+  const float* scal; int scal_base; int scal_mode;  // 0: none, 1: alpha^2, 2: alpha
+};
+cudaError_t launch_sgemm(const SgParams& p, cudaStream_t s);
+
+// ------------------------------------------------------------------ self-test
+cudaError_t launch_timeout_selftest(unsigned int* status, unsigned long long timeout_ns, cudaStream_t s);
+
+}  // namespace muon

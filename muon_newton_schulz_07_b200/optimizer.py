@@ -1,0 +1,84 @@
+"""PyTorch-facing wrapper of libmuon: torch allocates the workspace and provides the stream.
+
+    step = MuonStep([(1536, 1536), (1536, 6144), ...], dtype=torch.bfloat16)
+    step(W_list, G_list, M_list, lr=0.02, beta=0.95)      # W and M updated in place
+
+Only argument checking and pointer marshalling happen here; the optimizer step
+itself runs in libmuon's kernels on the current CUDA stream.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+QUINTIC = (3.4445, -4.7750, 2.0315)
+
+
+class MuonStep:
+    """A Muon step for one fixed list of matrix shapes, bound to one CUDA device."""
+
+    def __init__(self, shapes, dtype=torch.bfloat16, mode: str = "fast", device=None):
+        if dtype not in (torch.bfloat16, torch.float32):
+            raise TypeError("dtype must be torch.bfloat16 or torch.float32")
+        if mode not in ("fast", "fp32_ref"):
+            raise ValueError("mode must be 'fast' or 'fp32_ref'")
+        self.shapes = [(int(r), int(c)) for r, c in shapes]
+        self.dtype = dtype
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self._dt = B.MUON_BF16 if dtype == torch.bfloat16 else B.MUON_FP32
+        self._mode = B.MUON_MODE_FAST if mode == "fast" else B.MUON_MODE_FP32_REF
+        nbytes = B.muon_workspace_size(self.shapes, self._dt, self._mode)
+        self.workspace_bytes = nbytes
+        with torch.cuda.device(self.device):
+            self._ws = torch.empty(nbytes + 1024, dtype=torch.uint8, device=self.device)
+            base = self._ws.data_ptr()
+            self._ws_ptr = (base + 1023) // 1024 * 1024
+            self.handle = B.muon_create(self.shapes, self._dt, self._mode, self._ws_ptr, nbytes)
+        self.n_groups, _ = B.muon_get_plan(self.handle, 5)
+
+    def launches_per_step(self, ns_steps: int = 5) -> int:
+        return B.muon_get_plan(self.handle, ns_steps)[1]
+
+    def _check(self, tensors, name):
+        if len(tensors) != len(self.shapes):
+            raise ValueError(f"{name}: expected {len(self.shapes)} tensors, got {len(tensors)}")
+        for t, s in zip(tensors, self.shapes):
+            if tuple(t.shape) != s or t.dtype != self.dtype or t.device != self.device or not t.is_contiguous():
+                raise ValueError(f"{name}: tensor {tuple(t.shape)} {t.dtype} {t.device} does not match {s} "
+                                 f"{self.dtype} {self.device} (contiguous)")
+        return [t.data_ptr() for t in tensors]
+
+    def __call__(self, W, G, M, lr=0.02, beta=0.95, weight_decay=0.0, eps=1e-7, abc=QUINTIC, nesterov=True,
+                 ns_steps=5, stream=None):
+        hp = B.make_hparams(lr, beta, weight_decay, eps, abc, nesterov, ns_steps)
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        B.muon_step(self.handle, self._check(W, "W"), self._check(G, "G"), self._check(M, "M"), hp, s.cuda_stream)
+
+    def orthogonalize(self, X, O, eps=1e-7, abc=QUINTIC, ns_steps=5, stream=None):
+        hp = B.make_hparams(0.0, 0.0, 0.0, eps, abc, False, ns_steps)
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        B.muon_orthogonalize(self.handle, self._check(X, "X"), self._check(O, "O"), hp, s.cuda_stream)
+
+    def norms(self, out=None, stream=None) -> torch.Tensor:
+        """||U_i||_F of the last step, fp32, enqueued as one copy into `out` (device or pinned host)."""
+        if out is None:
+            out = torch.empty(len(self.shapes), dtype=torch.float32, device=self.device)
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        B.muon_get_norms(self.handle, out.data_ptr(), s.cuda_stream)
+        return out
+
+    def status(self, stream=None) -> int:
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        return B.muon_get_status(self.handle, s.cuda_stream)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            B.muon_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
