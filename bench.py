@@ -37,6 +37,8 @@ def parse():
     ap.add_argument("--impl", choices=["muon", "reference"], default="muon")
     ap.add_argument("--workload", default="d24", choices=["gpt2s", "d24", "l38b", "stress"])
     ap.add_argument("--ns-steps", type=int, default=5)
+    ap.add_argument("--matrices", type=int, default=0,
+                    help="use only the first N matrices of the workload (profiling captures of a smaller case)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-budget-s", type=float, default=150.0)
@@ -250,6 +252,10 @@ def run_muon(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = I.WORKLOADS[args.workload]
+    if args.matrices:
+        import dataclasses
+
+        wl = dataclasses.replace(wl, shapes=wl.shapes[:args.matrices], name=f"{wl.name}[:{args.matrices}]")
     shapes = list(wl.shapes)
     n = len(shapes)
     k = args.ns_steps

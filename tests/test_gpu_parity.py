@@ -104,16 +104,26 @@ def test_orthogonalize_shapes(mode, dtype, k):
     Xs_np = [rng.standard_normal(s).astype(np.float32) for s in SHAPES]
     Xs = [device_tensor(x, dtype) for x in Xs_np]
     Os = run_orthogonalize(SHAPES, Xs, dtype, mode, k=k)
-    # After one iteration the bf16 path has rounded U, A, B and X once each (<= 2^-9 relative
-    # apiece), so 8e-3 bounds it; further iterations are held to the 2e-2 budget.
-    tol = TOL_O[mode] if (mode == "fp32_ref" or k > 1) else 8e-3
-    tol += out_rounding(dtype)
+    a, b, c = O.QUINTIC
     errs = []
     for s, x, o in zip(SHAPES, Xs, Os):
-        ref = O.newton_schulz(to_f64(x), k, O.QUINTIC, 1e-7)
-        errs.append((rel_fro(to_f64(o), ref), s))
+        X = to_f64(x)
+        ref = O.newton_schulz(X, k, O.QUINTIC, 1e-7)
+        err = rel_fro(to_f64(o), ref)
+        if mode == "fast" and k == 1:
+            # One bf16 iteration rounds U, A, B and X once each (relative 2^-9 apiece).  B's
+            # rounding reaches X through a X + B X, where a + b s^2 + c s^4 can cancel: it is
+            # amplified by |b s^2 + c s^4| / |a + b s^2 + c s^4| at the largest normalised s.
+            smax = np.linalg.norm(X, 2) / np.linalg.norm(X)
+            y = smax * smax
+            amp = abs(b * y + c * y * y) / abs(a + b * y + c * y * y)
+            tol = 2.0 ** -9 * (3.0 + amp) * 1.25
+        else:
+            tol = TOL_O[mode]
+        tol += out_rounding(dtype)
+        errs.append((err, s))
+        assert err < tol, (s, err, tol)
     print(f"orthogonalize {mode} {dtype} k={k}: " + " ".join(f"{s[0]}x{s[1]}:{e:.2e}" for e, s in errs))
-    assert max(errs)[0] < tol, max(errs)
 
 
 def test_intermediates_symmetric_and_padded():
