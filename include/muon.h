@@ -172,6 +172,32 @@ MUON_API const char* muon_status_string(muon_status_t status);
 MUON_API muon_status_t muon_get_plan(muon_handle_t handle, int ns_steps, int* n_groups, int* launches_per_step);
 
 /*
+ * Momentum, Nesterov blend and Frobenius norm of ONE matrix, with no workspace.
+ * The pages have no counterpart for this entry point: it exists for callers that
+ * cannot give this library device memory (a framework whose allocator must own
+ * every device allocation, a fixed memory pool, code that may not call
+ * cudaMalloc).  It computes, for the rows x cols row-major matrix of `dtype`,
+ *   M <- beta*M + (1-beta)*G   (in place),
+ *   U <- (1-beta)*G + beta*M   if nesterov, else U <- M   (U: same shape/dtype),
+ *   *norm <- ||U||_F           (fp32; `norm` is a device pointer to one float),
+ * the same arithmetic as the first stage of muon_step (U in the caller's layout,
+ * not transposed).  The norm's reduction scratch is a fixed array of device
+ * memory inside libmuon.so (about 16 KB, held by every GPU that loads the
+ * library until the process exits); the call allocates nothing.
+ *   - rows * cols may be at most MUON_STATIC_MAX_ELEMENTS, else
+ *     MUON_ERR_UNSUPPORTED is returned and nothing is enqueued.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make it before capturing any stream.
+ *   - All calls share the array.  Calls in sequence on one stream are
+ *     independent (the arrival counter is cleared at the start of each call);
+ *     calls that overlap on the GPU race and give wrong norms.
+ */
+#define MUON_STATIC_MAX_ELEMENTS (1ll << 28)
+MUON_API muon_status_t muon_momentum_norm_static(const void* G, void* M, void* U, int64_t rows, int64_t cols,
+                                                 muon_dtype_t dtype, float beta, int32_t nesterov, float* norm,
+                                                 cudaStream_t stream);
+
+/*
  * Workspace introspection, for tests and tools.  muon_get_matrix_slot gives the
  * shape group of matrix i and its slot inside the group's batched buffers;
  * muon_get_group_buffers gives a group's padded oriented shape (mp x np, both

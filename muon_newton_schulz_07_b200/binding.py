@@ -207,3 +207,14 @@ def muon_get_group_buffers(handle: int, group: int):
     _check(lib().muon_get_group_buffers(handle, group, ctypes.byref(mp), ctypes.byref(np_), ctypes.byref(cnt),
                                         *[ctypes.byref(p) for p in ptrs]), "muon_get_group_buffers")
     return (mp.value, np_.value, cnt.value) + tuple(p.value for p in ptrs)
+
+
+def muon_momentum_norm_static(G: int, M: int, U: int, rows: int, cols: int, dtype: int, beta: float,
+                              nesterov: bool, norm: int, stream: int) -> None:
+    L = lib()
+    f = L.muon_momentum_norm_static
+    f.argtypes = [_VP, _VP, _VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_int32, _VP,
+                  _VP]
+    f.restype = ctypes.c_int
+    _check(f(ctypes.c_void_p(G), ctypes.c_void_p(M), ctypes.c_void_p(U), int(rows), int(cols), dtype, float(beta),
+             1 if nesterov else 0, ctypes.c_void_p(norm), ctypes.c_void_p(stream)), "muon_momentum_norm_static")
