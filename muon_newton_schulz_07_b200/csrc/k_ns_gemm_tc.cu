@@ -9,25 +9,36 @@
 // name for Muon's matrix parameters (aiproducthub "开发者千美元训3.8B模型 击败GPT-2",
 // 影响 paragraph).
 //
-// Gram and Poly outputs are symmetric: only 256 x 256 macro tiles on or above
-// the diagonal are computed (two 128-row CTA tiles each); every element on or
-// above the diagonal is stored at (r, c) and mirrored to (c, r), so the result
-// is exactly symmetric.
+// CTA pairs.  The kernel runs as clusters of two CTAs (one per SM of a TPC).
+// A pair computes one 256 x 256 output tile with tcgen05.mma.cta_group::2
+// (M = 256, N = 256, K = 16): CTA r holds rows 128r..128r+127 of the A operand
+// and half of the B operand (tile columns 128r..128r+127) in its own shared
+// memory, and rows 128r..128r+127 of the fp32 accumulator in its TMEM.  Each
+// CTA loads only its own halves (TMA, no multicast), so per k slice a CTA moves
+// 32 KB for 128 x 256 x 64 multiply-adds, two thirds of what a single-CTA
+// 128 x 256 tile needs.  The even CTA issues the MMAs; its commits are
+// multicast to the barriers of both CTAs.
 //
-// CTA layout (192 threads, one CTA per SM, persistent over a static
-// round-robin tile list):
-//   warp 0      TMA producer: 64 x 64 bf16 boxes, 128-byte swizzle, into a
-//               4-stage ring of {A 128 x 64, B 256 x 64} shared-memory tiles
-//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f16,
-//               M = 128, N = 256, K = 16, fp32 accumulators in TMEM, two
-//               accumulator buffers (2 x 256 columns) so the epilogue of one
-//               tile overlaps the main loop of the next
+// Gram and Poly outputs are symmetric: only 256 x 256 tiles on or above the
+// diagonal are computed; every element on or above the diagonal is stored at
+// (r, c) and mirrored to (c, r), so the result is exactly symmetric.
+//
+// Roles in each CTA (192 threads, one CTA per SM, persistent over a static
+// round-robin list of pair tiles):
+//   warp 0      TMA producer into a 6-stage ring of {A 128 x 64, B 128 x 64}
+//               bf16 tiles (64 x 64 boxes, 128-byte swizzle); the even CTA's
+//               full barrier counts the bytes of both CTAs
+//   warp 1      TMEM allocation (512 columns: two 256-column accumulators, so
+//               the epilogue of one tile overlaps the main loop of the next);
+//               in the even CTA, lane 0 issues the MMAs
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, the fp32 combination
 //               with the auxiliary input (A for Poly, X for Update), bf16 cast,
 //               global stores (plus the mirrored store for Gram/Poly)
 // Operand B of Update is X itself in its row-major layout, i.e. MN-major; the
 // other operands are K-major.  All waits are bounded (see muon_device.cuh).
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "muon_device.cuh"
 #include "muon_internal.h"
@@ -36,10 +47,11 @@ namespace muon {
 namespace {
 
 constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK, STAGES = kTcStages;
+constexpr int TILE = 256;                               // pair tile: 256 x 256
 constexpr uint32_t BOX_BYTES = 64 * 64 * 2;             // one TMA box
-constexpr uint32_t A_STAGE = BM * BK * 2;               // 16 KB
-constexpr uint32_t B_STAGE = BN * BK * 2;               // 32 KB
-constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE;     // 48 KB
+constexpr uint32_t A_STAGE = BM * BK * 2;               // 16 KB: this CTA's 128 rows of A
+constexpr uint32_t B_STAGE = (BN / 2) * BK * 2;         // 16 KB: this CTA's half of B
+constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE;     // 32 KB
 constexpr uint32_t TMEM_COLS = 512;                     // 2 accumulators x 256 fp32 columns
 constexpr uint32_t BAR_BYTES = 256;
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
@@ -60,17 +72,17 @@ __device__ __forceinline__ Tile decode_tile(const TcParams& p, int t) {
   ti.mat = mat;
   if (p.kind == kUpdate) {
     const int tm = r / G.tdim;
-    ti.row0 = tm * BM;
-    ti.col0 = (r - tm * G.tdim) * BN;
+    ti.row0 = tm * TILE;
+    ti.col0 = (r - tm * G.tdim) * TILE;
   } else {
-    // upper-triangle macro tile q = (I, J), I <= J, row-major; two row halves each
-    int q = r >> 1, I = 0;
+    // upper-triangle tile q = (I, J), I <= J, row-major over the triangle
+    int q = r, I = 0;
     while (q >= G.tdim - I) {
       q -= G.tdim - I;
       ++I;
     }
-    ti.row0 = I * 256 + (r & 1) * BM;
-    ti.col0 = (I + q) * 256;
+    ti.row0 = I * TILE;
+    ti.col0 = (I + q) * TILE;
   }
   return ti;
 }
@@ -92,7 +104,8 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
   return q;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1) ns_gemm_tc_kernel(const __grid_constant__ TcParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+    ns_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t smem_base = smem_u32(smem);
@@ -106,15 +119,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) ns_gemm_tc_kernel(const __grid_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();           // 0: issues the MMAs; 1: its peer
+  const int cl = static_cast<int>(cluster_id_x());
+  const int ncl = static_cast<int>(num_clusters_x());
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(full_bar(s), 1);   // the even CTA's arrive.expect_tx (bytes of both CTAs)
+      mbar_init(empty_bar(s), 1);  // one multicast commit
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(accf_bar(a), 1);
-      mbar_init(acce_bar(a), 4);  // one arrival per epilogue warp
+      mbar_init(accf_bar(a), 1);   // one multicast commit
+      mbar_init(acce_bar(a), 8);   // one arrival per epilogue warp of both CTAs
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -126,41 +142,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) ns_gemm_tc_kernel(const __grid_
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_arrive_wait();  // barriers of both CTAs initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t tmo = p.timeout_ns;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------------------------------------------------- TMA producer
+      // ---------------------------------------------------------- TMA producer (both CTAs)
       int stage = 0;
       uint32_t phase = 0;
-      for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+      const int half = static_cast<int>(rank) * (BN / 2);
+      for (int t = cl; t < p.total_tiles; t += ncl) {
         const Tile ti = decode_tile(p, t);
         const TcGroup& G = p.g[ti.g];
+        const int arow = ti.row0 + static_cast<int>(rank) * BM;
         bool ok = true;
         for (int kb = 0; kb < G.kblocks; ++kb) {
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          const uint32_t fb = map_to_rank(full_bar(stage), 0);
           const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + A_STAGE;
           const int k0 = kb * BK;
-          tma_load_3d(sa, &G.tm_a, fb, k0, ti.row0, ti.mat);
-          tma_load_3d(sa + BOX_BYTES, &G.tm_a, fb, k0, ti.row0 + 64, ti.mat);
+          tma_load_3d_pair(sa, &G.tm_a, fb, k0, arow, ti.mat);
+          tma_load_3d_pair(sa + BOX_BYTES, &G.tm_a, fb, k0, arow + 64, ti.mat);
           if (p.kind != kUpdate) {
-#pragma unroll
-            for (int h = 0; h < 4; ++h) tma_load_3d(sb + h * BOX_BYTES, &G.tm_b, fb, k0, ti.col0 + 64 * h, ti.mat);
+            tma_load_3d_pair(sb, &G.tm_b, fb, k0, ti.col0 + half, ti.mat);
+            tma_load_3d_pair(sb + BOX_BYTES, &G.tm_b, fb, k0, ti.col0 + half + 64, ti.mat);
           } else {
-#pragma unroll
-            for (int h = 0; h < 4; ++h) tma_load_3d(sb + h * BOX_BYTES, &G.tm_b, fb, ti.col0 + 64 * h, k0, ti.mat);
+            tma_load_3d_pair(sb, &G.tm_b, fb, ti.col0 + half, k0, ti.mat);
+            tma_load_3d_pair(sb + BOX_BYTES, &G.tm_b, fb, ti.col0 + half + 64, k0, ti.mat);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -169,8 +187,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) ns_gemm_tc_kernel(const __grid_
         }
         if (!ok) break;
       }
-      // Do not leave the CTA while loads are still landing in shared memory:
-      // wait (bounded) until every stage's last armed phase has completed.
+      // Do not leave while loads or MMAs may still touch this CTA's shared memory:
+      // wait (bounded) until the last use of every stage has been released.
       for (int i = 0; i < STAGES; ++i) {
         if (*abort_flag) break;
         (void)mbar_wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, p.status);
@@ -181,15 +199,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) ns_gemm_tc_kernel(const __grid_
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, p.kind == kUpdate ? 1 : 0);
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------- MMA issuer (even CTA)
+      const uint32_t idesc = idesc_bf16_f32(2 * BM, BN, 0, p.kind == kUpdate ? 1 : 0);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+      for (int t = cl; t < p.total_tiles && ok; t += ncl) {
         const Tile ti = decode_tile(p, t);
         const TcGroup& G = p.g[ti.g];
         if (!mbar_wait_bounded(acce_bar(acc), acc_phase ^ 1u, tmo, abort_flag, p.status)) break;
@@ -207,27 +225,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) ns_gemm_tc_kernel(const __grid_
             const uint64_t adesc = smem_desc_sw128(sa + 32u * j, 16, 1024);
             const uint64_t bdesc = (p.kind == kUpdate) ? smem_desc_sw128(sb + 2048u * j, 8192, 1024)
                                                        : smem_desc_sw128(sb + 32u * j, 16, 1024);
-            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | j) != 0 ? 1u : 0u);
+            tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | j) != 0 ? 1u : 0u);
           }
-          tc_commit(empty_bar(stage));  // frees the stage once these MMAs have read it
+          tc_commit_pair_mc(empty_bar(stage), 0x3);  // frees the stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(accf_bar(acc));  // accumulator ready for the epilogue
+        tc_commit_pair_mc(accf_bar(acc), 0x3);  // accumulator ready for both epilogues
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
-    const int row_in_tile = quad * 32 + lane;
+    const int row_in_tile = static_cast<int>(rank) * BM + quad * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+    for (int t = cl; t < p.total_tiles; t += ncl) {
       const Tile ti = decode_tile(p, t);
       const TcGroup& G = p.g[ti.g];
       if (!mbar_wait_bounded(accf_bar(acc), acc_phase, tmo, abort_flag, p.status)) break;
@@ -243,16 +261,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) ns_gemm_tc_kernel(const __grid_
       const __nv_bfloat16* aux = G.aux ? static_cast<const __nv_bfloat16*>(G.aux) + mat_off : nullptr;
       const int gr = ti.row0 + row_in_tile;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t acce_leader = map_to_rank(acce_bar(acc), 0);
 #pragma unroll 1
       for (int ch = 0; ch < BN / 32; ++ch) {
         float v[32];
         __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the divergent stores below
         tmem_ld_32cols(taddr + ch * 32, v);
         if (ch == BN / 32 - 1) {
-          // all of this accumulator has been read: hand it back to the MMA warp
+          // all of this accumulator has been read: hand it back to the MMA issuer
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(acce_bar(acc));
+          if (lane == 0) mbar_arrive_remote(acce_leader);
         }
         const int gc0 = ti.col0 + ch * 32;
         const bool symmetric = (p.kind != kUpdate);
@@ -295,10 +314,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) ns_gemm_tc_kernel(const __grid_
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  cluster_arrive_wait();  // neither CTA frees TMEM or leaves while the pair may still use it
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -315,8 +335,9 @@ cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-  ns_gemm_tc_kernel<<<grid, kTcThreads, SMEM_BYTES, s>>>(p);
+  // one CTA pair per TPC, at most one pair per tile
+  const int pairs = std::min(num_sms / 2, p.total_tiles);
+  ns_gemm_tc_kernel<<<2 * pairs, kTcThreads, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -336,7 +336,7 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_b = gp.tm_x[cur];
               G.out = h->ws + gp.off_a;
               G.aux = nullptr;
-              G.tiles_per_mat = T * (T + 1);
+              G.tiles_per_mat = T * (T + 1) / 2;  // 256 x 256 pair tiles on or above the diagonal
               G.kblocks = gp.np / kTcBK;
               G.tdim = T;
               G.out_ld = gp.mp;
@@ -345,7 +345,7 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_b = gp.tm_a;
               G.out = h->ws + gp.off_b;
               G.aux = h->ws + gp.off_a;
-              G.tiles_per_mat = T * (T + 1);
+              G.tiles_per_mat = T * (T + 1) / 2;
               G.kblocks = gp.mp / kTcBK;
               G.tdim = T;
               G.out_ld = gp.mp;
@@ -354,9 +354,9 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_b = gp.tm_x[cur];
               G.out = h->ws + gp.off_x[nxt];
               G.aux = h->ws + gp.off_x[cur];
-              G.tiles_per_mat = (gp.mp / kTcBM) * (gp.np / kTcBN);
+              G.tiles_per_mat = (gp.mp / 256) * (gp.np / 256);  // 256 x 256 pair tiles
               G.kblocks = gp.mp / kTcBK;
-              G.tdim = gp.np / kTcBN;
+              G.tdim = gp.np / 256;
               G.out_ld = gp.np;
             }
             tiles += G.tiles_per_mat * gp.cnt;

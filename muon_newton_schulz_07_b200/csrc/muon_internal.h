@@ -85,7 +85,7 @@ cudaError_t launch_param_write(const WrParams& p, Dtype io, Dtype xt, cudaStream
 constexpr int kTcBM = 128;
 constexpr int kTcBN = 256;
 constexpr int kTcBK = 64;
-constexpr int kTcStages = 4;
+constexpr int kTcStages = 6;
 constexpr int kTcMaxGroups = 6;
 constexpr int kTcThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 

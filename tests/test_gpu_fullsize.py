@@ -1,0 +1,157 @@
+"""Parity at full size, in the launch configuration bench.py times (one MuonStep over the whole set).
+
+The oracle cannot step 144-168 matrices of these sizes in seconds, so it checks sampled matrices:
+the first, middle and last matrix of each distinct shape.  The orthogonalised direction is read
+from the workspace (the final iterate X_k of the step, oriented min x max), and M1 and W1 from the
+caller's tensors.  The conditioning-stress set is checked against the scalar polynomial, singular
+value by singular value.
+"""
+from __future__ import annotations
+
+import math
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from muon_newton_schulz_07_b200 import binding as B
+from muon_newton_schulz_07_b200 import inputs as I
+from muon_newton_schulz_07_b200.optimizer import MuonStep
+
+from helpers import bf16_ulp, rel_fro, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def gen_all(fn, n):
+    with ThreadPoolExecutor(16) as ex:
+        return [torch.from_numpy(a).cuda().to(torch.bfloat16) for a in ex.map(fn, range(n))]
+
+
+def final_iterate(op, i, k):
+    """X_k of matrix i as the step left it in the workspace (oriented: min x max)."""
+    g, slot = B.muon_get_matrix_slot(op.handle, i)
+    mp, np_, _, x0, x1, _, _ = B.muon_get_group_buffers(op.handle, g)
+    base = (x0, x1)[k & 1]
+    off = base - op._ws.data_ptr() + slot * mp * np_ * 2
+    return op._ws[off:off + mp * np_ * 2].view(torch.bfloat16).view(mp, np_)
+
+
+def samples(shapes):
+    by = {}
+    for i, s in enumerate(shapes):
+        by.setdefault(s, []).append(i)
+    out = []
+    for s, idx in by.items():
+        out += sorted({idx[0], idx[len(idx) // 2], idx[-1]})
+    return out
+
+
+@pytest.mark.parametrize("name", ["d24", "l38b", "gpt2s"])
+def test_full_set_step_sampled(name):
+    wl = I.WORKLOADS[name]
+    n = len(wl.shapes)
+    W = gen_all(lambda i: I.weight(wl, i), n)
+    G = gen_all(lambda i: I.gradient(wl, 1, i), n)
+    M = gen_all(lambda i: I.momentum(wl, i), n)
+    check = samples(wl.shapes)
+    pre = {i: (to_f64(W[i]), to_f64(G[i]), to_f64(M[i])) for i in check}
+    op = MuonStep(wl.shapes, dtype=torch.bfloat16)
+    op(W, G, M, lr=0.02, beta=0.95, weight_decay=0.0, ns_steps=5)
+    torch.cuda.synchronize()
+    assert op.status() == B.MUON_OK
+    hp = O.Hyper(lr=0.02, beta=0.95, weight_decay=0.0, eps=1e-7, nesterov=True, ns_steps=5)
+    worst = 0.0
+    for i in check:
+        r, c = wl.shapes[i]
+        W0, G0, M0 = pre[i]
+        W1r, M1r, Or = O.muon_step(W0, G0, M0, hp)
+        m, nn = min(r, c), max(r, c)
+        Xk = to_f64(final_iterate(op, i, 5))
+        O_gpu = Xk[:m, :nn] if r <= c else Xk[:m, :nn].T
+        err = rel_fro(O_gpu, Or)
+        worst = max(worst, err)
+        assert err < 2e-2, (name, i, (r, c), err)
+        assert rel_fro(to_f64(M[i]), M1r) < 2.0 ** -8, (name, i)
+        bound = 0.5 * 1.01 * np.linalg.norm(bf16_ulp(W1r)) + 0.02 * O.shape_scale(r, c) * 2e-2 * np.linalg.norm(Or)
+        assert np.linalg.norm(to_f64(W[i]) - W1r) <= bound, (name, i)
+        # the padding of the workspace stays zero
+        assert not Xk[m:, :].any() and not Xk[:, nn:].any()
+    print(f"{name}: {len(check)} sampled matrices, worst O error {worst:.3e}")
+    op.close()
+
+
+STRESS_IDX = [0, 1, 64, 65, 128, 129, 192, 193]  # two matrices of each stress shape, full size
+
+# Largest value of the quintic on [0, 1]: normalised singular values start in [0, 1] and
+# the iteration keeps them in [0, PHI_MAX] (the polynomial has no real root there).
+PHI_MAX = 1.2024
+
+
+def linear_gain(x, k, abc=O.QUINTIC):
+    """|d phi^k / dx| along the scalar trajectory (chain rule)."""
+    a, b, c = abc
+    g = np.ones_like(x)
+    for _ in range(k):
+        g = g * np.abs(a + 3 * b * x * x + 5 * c * x ** 4)
+        x = a * x + b * x ** 3 + c * x ** 5
+    return g
+
+
+def stress_run(mode, dtype, k):
+    wl = I.WORKLOADS["stress"]
+    shapes = [wl.shapes[i] for i in STRESS_IDX]
+    X = [torch.from_numpy(I.momentum(wl, i)).cuda().to(dtype) for i in STRESS_IDX]
+    Os = [torch.empty_like(x) for x in X]
+    op = MuonStep(shapes, dtype=dtype, mode=mode)
+    op.orthogonalize(X, Os, ns_steps=k)
+    torch.cuda.synchronize()
+    assert op.status() == B.MUON_OK
+    op.close()
+    for x, o, s in zip(X, Os, shapes):
+        U = to_f64(x)
+        P, sv, Qt = np.linalg.svd(U, full_matrices=False)
+        xs = sv / (math.sqrt(float(np.sum(sv * sv))) + 1e-7)
+        yield s, U, to_f64(o), P, xs, Qt
+
+
+@pytest.mark.parametrize("k", [5, 10])
+def test_stress_fp32_reference_mode(k):
+    # Condition numbers up to 1e6: the fp32 mode meets the oracle at 1e-4 even after 10 steps,
+    # and D = P^T O Q (SVD of the input, fp64) is diagonal with the scalar polynomial's values.
+    for s, U, Og, P, xs, Qt in stress_run("fp32_ref", torch.float32, k):
+        ref = O.newton_schulz(U, k)
+        err = rel_fro(Og, ref)
+        D = P.T @ Og @ Qt.T
+        diag_err = np.max(np.abs(np.diag(D) - O.scalar_map(xs, k)))
+        off = np.linalg.norm(D - np.diag(np.diag(D))) / np.linalg.norm(D)
+        print(f"stress fp32_ref {s} k={k}: vs oracle {err:.2e}, diag {diag_err:.2e}, off-diagonal {off:.2e}")
+        assert err < 1e-4, (s, err)
+        assert diag_err < 1e-4 * max(1.0, np.linalg.norm(D)) and off < 1e-4, (s, diag_err, off)
+
+
+@pytest.mark.parametrize("k", [5, 10])
+def test_stress_bf16_singular_value_map(k):
+    # bf16 operands round X, A and B to 8 bits: by Weyl's inequality each rounding of the
+    # normalised X moves every singular value by at most u = 2^-9, and k steps amplify an
+    # input perturbation of direction i by the gain of phi^k at s_i.  Directions with
+    # gain * u <= 1e-2 are resolvable; on them D = P^T O Q must follow the scalar
+    # polynomial (3e-2) and O must match the oracle (2e-2).  Every direction, resolvable or
+    # not, stays inside the quintic's invariant band [0, PHI_MAX] (to bf16 accuracy).
+    u = 2.0 ** -9
+    for s, U, Og, P, xs, Qt in stress_run("fast", torch.bfloat16, k):
+        ok = linear_gain(xs, k) * u <= 1e-2
+        Pr, Qr = P[:, ok], Qt[ok, :].T
+        D = Pr.T @ Og @ Qr
+        diag_err = np.max(np.abs(np.diag(D) - O.scalar_map(xs[ok], k))) if ok.any() else 0.0
+        ref = O.newton_schulz(U, k)
+        sub_err = rel_fro(Pr.T @ Og @ Qr, Pr.T @ ref @ Qr) if ok.any() else 0.0
+        top = np.linalg.norm(Og, 2)
+        print(f"stress bf16 {s} k={k}: {ok.sum()}/{len(xs)} resolvable, diag {diag_err:.2e}, "
+              f"resolvable-subspace error {sub_err:.2e}, ||O||_2 {top:.4f}")
+        assert ok.sum() >= 16, (s, ok.sum())
+        assert diag_err < 3e-2, (s, diag_err)
+        assert sub_err < 2e-2, (s, sub_err)
+        assert top <= PHI_MAX * (1 + 4 * u), (s, top)
