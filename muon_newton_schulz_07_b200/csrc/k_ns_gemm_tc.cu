@@ -3,11 +3,13 @@
 // One persistent kernel runs one stage of one Newton-Schulz iteration for every
 // matrix of the parameter set (all shape groups in one launch):
 //   Gram    A = s * X X^T          (s = 1/(||U||+eps)^2 on the first iteration)
-//   Poly    B = b * A + c * A A    (A symmetric, so A A = A A^T)
-//   Update  X' = s * (a * X + B X) (s = 1/(||U||+eps) on the first iteration)
+//   Poly    B' = a I + b A + c A A (A symmetric, so A A = A A^T)
+//   Update  X' = s * (B' X)        (s = 1/(||U||+eps) on the first iteration)
 // which together are one step of the Newton-Schulz orthogonalisation the pages
 // name for Muon's matrix parameters (aiproducthub "开发者千美元训3.8B模型 击败GPT-2",
-// 影响 paragraph).
+// 影响 paragraph).  B' carries the a X term of the update (a X + B X =
+// (a I + B) X), which also keeps the cancellation a + b s^2 + c s^4 inside one
+// fp32 sum before rounding.
 //
 // CTA pairs.  The kernel runs as clusters of two CTAs (one per SM of a TPC).
 // A pair computes one 256 x 256 output tile with tcgen05.mma.cta_group::2
@@ -32,8 +34,12 @@
 //               the epilogue of one tile overlaps the main loop of the next);
 //               in the even CTA, lane 0 issues the MMAs
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, the fp32 combination
-//               with the auxiliary input (A for Poly, X for Update), bf16 cast,
-//               global stores (plus the mirrored store for Gram/Poly)
+//               (Poly: c A A + b A + a I), bf16 cast, stores staged through
+//               shared memory so every global access is a 64-byte row run
+//               (plus the mirrored store for Gram/Poly).  In the last Update
+//               the epilogue writes the parameters directly:
+//               W = (1 - lr wd) W - lr sqrt(max(1, r/c)) X_k from the unrounded
+//               fp32 X_k, transposed back for tall matrices.
 // Operand B of Update is X itself in its row-major layout, i.e. MN-major; the
 // other operands are K-major.  All waits are bounded (see muon_device.cuh).
 #include <cuda_bf16.h>
@@ -54,7 +60,12 @@ constexpr uint32_t B_STAGE = (BN / 2) * BK * 2;         // 16 KB: this CTA's hal
 constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE;     // 32 KB
 constexpr uint32_t TMEM_COLS = 512;                     // 2 accumulators x 256 fp32 columns
 constexpr uint32_t BAR_BYTES = 256;
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+constexpr int EPI_PITCH = 40;                            // staged row: 32 bf16 + 8 pad (80 B, 16-B aligned)
+constexpr int F32_PITCH = 36;                            // staged fp32 row: 32 + 4 pad (144 B, 16-B aligned)
+constexpr uint32_t EPI_WARP_BYTES = 2 * 32 * EPI_PITCH * 2;  // output + auxiliary chunk per warp
+constexpr uint32_t EPI_OFFSET = STAGES * STAGE_BYTES + BAR_BYTES;
+constexpr size_t SMEM_BYTES = 1024 + EPI_OFFSET + 4 * EPI_WARP_BYTES;
+static_assert(32 * F32_PITCH * 4 <= EPI_WARP_BYTES, "fp32 staging must fit the per-warp buffer");
 
 struct Tile {
   int g, mat, row0, col0;
@@ -241,13 +252,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    // Each warp owns 32 rows of the CTA's 128 (its TMEM lane quadrant) and walks the tile
+    // in 32 x 32 chunks.  A chunk goes through a per-warp shared staging buffer so that
+    // every global access is a run of 64 contiguous bytes: 8 rows x 4 lanes x 16 bytes
+    // per instruction (the auxiliary input, the direct store and the mirrored store).
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
-    const int row_in_tile = static_cast<int>(rank) * BM + quad * 32 + lane;
+    __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + EPI_OFFSET + (warp - 2) * EPI_WARP_BYTES);
+    __nv_bfloat16* stg_aux = stg + 32 * EPI_PITCH;
+    const int sub_r = lane >> 2, sub_c = (lane & 3) * 8;
+    const bool symmetric = (p.kind != kUpdate);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = cl; t < p.total_tiles; t += ncl) {
       const Tile ti = decode_tile(p, t);
       const TcGroup& G = p.g[ti.g];
+      const int ld = G.out_ld;
+      const size_t mat_off = static_cast<size_t>(ti.mat) * G.mp * ld;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(G.out) + mat_off;
+      const __nv_bfloat16* aux = G.aux ? static_cast<const __nv_bfloat16*>(G.aux) + mat_off : nullptr;
+      const int gr0 = ti.row0 + static_cast<int>(rank) * BM + quad * 32;  // first row of this warp
+      const int gr = gr0 + lane;
+      // The auxiliary input does not depend on the accumulator: fetch its first chunk
+      // (the first one at or above the diagonal) before waiting, and every later chunk
+      // one step ahead, so its latency hides behind the accumulator drain.
+      uint4 pf[4];
+      auto aux_load = [&](int c, uint4 (&dst)[4]) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = __ldg(reinterpret_cast<const uint4*>(aux + static_cast<size_t>(gr0 + q * 8 + sub_r) * ld +
+                                                        ti.col0 + c * 32 + sub_c));
+      };
+      if (aux != nullptr) {
+        int c0 = 0;
+        while (symmetric && c0 < BN / 32 - 1 && ti.col0 + c0 * 32 + 32 <= gr0) ++c0;
+        aux_load(c0, pf);
+      }
       if (!mbar_wait_bounded(accf_bar(acc), acc_phase, tmo, abort_flag, p.status)) break;
       tc_fence_after();
       float s = 1.0f;
@@ -255,33 +294,92 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         const float al = p.scal[2 * (G.scal_base + ti.mat) + 1];
         s = (p.kind == kGram) ? al * al : al;
       }
-      const int ld = G.out_ld;
-      const size_t mat_off = static_cast<size_t>(ti.mat) * G.mp * ld;
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(G.out) + mat_off;
-      const __nv_bfloat16* aux = G.aux ? static_cast<const __nv_bfloat16*>(G.aux) + mat_off : nullptr;
-      const int gr = ti.row0 + row_in_tile;
+      const float cdiag = (p.kind == kPoly && gr < G.m_real) ? p.c_diag : 0.0f;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const uint32_t acce_leader = map_to_rank(acce_bar(acc), 0);
 #pragma unroll 1
       for (int ch = 0; ch < BN / 32; ++ch) {
+        const int gc0 = ti.col0 + ch * 32;
+        // Chunks of Gram/Poly tiles lie fully above the diagonal, on it, or fully below it
+        // (rows and columns are both multiples of 32); the ones below are mirrored from
+        // elsewhere.  The last chunk of a tile is never below the diagonal.
+        const bool below = symmetric && gc0 + 32 <= gr0;
+        const bool diag = symmetric && gc0 == gr0;
         float v[32];
-        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the divergent stores below
-        tmem_ld_32cols(taddr + ch * 32, v);
+        if (!below) {
+          __syncwarp();
+          tmem_ld_32cols(taddr + ch * 32, v);
+        }
         if (ch == BN / 32 - 1) {
           // all of this accumulator has been read: hand it back to the MMA issuer
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_remote(acce_leader);
         }
-        const int gc0 = ti.col0 + ch * 32;
-        const bool symmetric = (p.kind != kUpdate);
-        if (symmetric && gc0 + 31 < gr) continue;  // strictly below the diagonal: mirrored from elsewhere
+        if (below) continue;
+        if (p.fuse_write) {
+          // Last Update: write the parameters instead of X_k.  Chunks in the zero padding
+          // of the workspace have no parameters (real dimensions are multiples of 32).
+          if (gr0 >= G.m_real || gc0 >= G.n_real) continue;
+          const int slot = G.scal_base + ti.mat;
+          __nv_bfloat16* W = static_cast<__nv_bfloat16*>(p.wptr[slot]);
+          const float cw = p.wcoef[slot];
+          const bool tr = p.wtrans[slot] != 0;
+          const int ldw = tr ? G.m_real : G.n_real;
+          // element (row rr, 8 columns from sub_c) of this chunk in W's own layout
+          auto woff = [&](int rr) -> size_t {
+            return tr ? static_cast<size_t>(gc0 + rr) * ldw + gr0 + sub_c
+                      : static_cast<size_t>(gr0 + rr) * ldw + gc0 + sub_c;
+          };
+          uint4 wv[4];
+          if (p.w_decay != 0.0f) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) wv[q] = __ldcs(reinterpret_cast<const uint4*>(W + woff(q * 8 + sub_r)));
+          }
+          // stage s * acc in fp32 (row-major, or transposed for tall parameters)
+          float* st32 = reinterpret_cast<float*>(stg);
+          if (!tr) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(st32 + lane * F32_PITCH + i) =
+                  make_float4(s * v[i], s * v[i + 1], s * v[i + 2], s * v[i + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) st32[i * F32_PITCH + lane] = s * v[i];
+          }
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int rr = q * 8 + sub_r;
+            const float4 o0 = *reinterpret_cast<const float4*>(st32 + rr * F32_PITCH + sub_c);
+            const float4 o1 = *reinterpret_cast<const float4*>(st32 + rr * F32_PITCH + sub_c + 4);
+            float r8[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+            if (p.w_decay != 0.0f) {
+              float w8[8];
+              unpack8(wv[q], w8);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) r8[i] = fmaf(p.w_decay, w8[i], cw * r8[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) r8[i] = cw * r8[i];
+            }
+            __stcs(reinterpret_cast<uint4*>(W + woff(rr)), pack8(r8));
+          }
+          __syncwarp();
+          continue;
+        }
         if (aux != nullptr) {
-          const uint4* ap = reinterpret_cast<const uint4*>(aux + static_cast<size_t>(gr) * ld + gc0);
+          uint4 nx[4];
+          if (ch + 1 < BN / 32) aux_load(ch + 1, nx);  // a chunk after a non-skipped one is never skipped
+#pragma unroll
+          for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(stg_aux + (q * 8 + sub_r) * EPI_PITCH + sub_c) = pf[q];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) pf[q] = nx[q];
+          __syncwarp();
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float a8[8];
-            unpack8(__ldg(ap + q), a8);
+            unpack8(*reinterpret_cast<const uint4*>(stg_aux + lane * EPI_PITCH + q * 8), a8);
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[8 * q + i] = s * fmaf(p.c_acc, v[8 * q + i], p.c_aux * a8[i]);
           }
@@ -289,21 +387,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = s * p.c_acc * v[i];
         }
-        __nv_bfloat16* orow = out + static_cast<size_t>(gr) * ld + gc0;
-        if (!symmetric || gc0 >= gr) {
-          uint4* op = reinterpret_cast<uint4*>(orow);
+        if (diag) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) op[q] = pack8(v + 8 * q);
-        } else {
+          for (int i = 0; i < 32; ++i)
+            if (gc0 + i == gr) v[i] += cdiag;
+          // on-diagonal chunk: element-wise, keeping (r, c) with c >= r and mirroring c > r
+          __nv_bfloat16* orow = out + static_cast<size_t>(gr) * ld + gc0;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (gc0 + i >= gr) orow[i] = __float2bfloat16_rn(v[i]);
-        }
-        if (symmetric) {
-          // mirrored store: lanes hold consecutive rows, so each column store is coalesced
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (gc0 + i > gr) out[static_cast<size_t>(gc0 + i) * ld + gr] = __float2bfloat16_rn(v[i]);
+          continue;
+        }
+        // direct store: row-major staging, then 64-byte row runs
+#pragma unroll
+        for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(stg + lane * EPI_PITCH + q * 8) = pack8(v + 8 * q);
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int rr = q * 8 + sub_r;
+          *reinterpret_cast<uint4*>(out + static_cast<size_t>(gr0 + rr) * ld + gc0 + sub_c) =
+              *reinterpret_cast<const uint4*>(stg + rr * EPI_PITCH + sub_c);
+        }
+        if (symmetric) {
+          // mirrored store: transposed staging, then 64-byte runs of the mirrored rows
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) stg[i * EPI_PITCH + lane] = __float2bfloat16_rn(v[i]);
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int cc = q * 8 + sub_r;
+            *reinterpret_cast<uint4*>(out + static_cast<size_t>(gc0 + cc) * ld + gr0 + sub_c) =
+                *reinterpret_cast<const uint4*>(stg + cc * EPI_PITCH + sub_c);
+          }
         }
       }
       acc ^= 1;

@@ -1,8 +1,13 @@
 // FP32 reference-mode products of the Newton-Schulz iteration on the CUDA
-// cores: true fp32 FMA (no TF32), one batched launch per shape group and stage.
+// cores, one batched launch per shape group and stage.  Operands and results are
+// fp32; the products of fp32 numbers are exact in fp64 and are summed in fp64
+// (DFMA) and combined in fp64, so the only roundings are the fp32 stores of X, A
+// and B'.  (Summing in
+// fp32 along K = 8192 loses enough that ten Newton-Schulz steps, which amplify
+// small singular directions by up to a^10, miss 1e-4 on condition-1e6 inputs.)
 //   Gram:    C = s * (X X^T)           (b_trans = 1, second operand X itself)
-//   Poly:    C = c * (A A) + b * A     (A symmetric)
-//   Update:  C = s * (B X + a * X)
+//   Poly:    C = c * (A A) + b * A + a * I   (A symmetric; B' carries the a X term)
+//   Update:  C = s * (B' X)
 // 64 x 64 output tiles, 16-deep k slices through shared memory, 4 x 4 outputs per
 // thread.  Every dimension is a multiple of 64 (the workspace is zero-padded), so
 // the kernel has no edge predicates; the host checks this before launching.
@@ -25,11 +30,11 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const SgParams p) {
   float* C = p.c + z * p.sc;
   const int m0 = blockIdx.y * SB, n0 = blockIdx.x * SB;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4];
+  double acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
 
   for (int k0 = 0; k0 < p.K; k0 += SK) {
 #pragma unroll
@@ -46,7 +51,7 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const SgParams p) {
     __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < SK; ++kk) {
-      float a[4], b[4];
+      double a[4], b[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
 #pragma unroll
@@ -54,14 +59,15 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const SgParams p) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
     }
     __syncthreads();
   }
 
-  float s = 1.0f;
+  // The epilogue works in fp64 as well, so each stored element is rounded to fp32 once.
+  double s = 1.0;
   if (p.scal_mode != 0) {
-    const float al = p.scal[2 * (p.scal_base + z) + 1];
+    const double al = p.scal[2 * (p.scal_base + z) + 1];
     s = (p.scal_mode == 1) ? al * al : al;
   }
   const float* aux = p.aux ? p.aux + z * p.sc : nullptr;
@@ -71,9 +77,10 @@ __global__ void __launch_bounds__(256) sgemm_kernel(const SgParams p) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int col = n0 + tx * 4 + j;
-      float v = p.c_acc * acc[i][j];
-      if (aux) v = fmaf(p.c_aux, aux[row + col], v);
-      C[row + col] = s * v;
+      double v = static_cast<double>(p.c_acc) * acc[i][j];
+      if (aux) v = fma(static_cast<double>(p.c_aux), static_cast<double>(aux[row + col]), v);
+      if (col == m0 + ty * 4 + i && col < p.diag_n) v += p.c_diag;
+      C[row + col] = static_cast<float>(s * v);
     }
   }
 }

@@ -8,8 +8,9 @@
 //   momentum_norm_kernel   (one launch per <= 192 matrices)
 //   k x { Gram, Poly, Update }   tcgen05 kernels, every shape group in one launch
 //                                (or fp32 CUDA-core kernels, one per group, in
-//                                the reference mode)
-//   param_write_kernel     (one launch per <= 192 matrices)
+//                                the reference mode); the last Update writes the
+//                                parameters itself when the shapes allow it
+//   param_write_kernel     (one launch per <= 192 matrices, only when not fused)
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
@@ -113,7 +114,8 @@ void make_plan(const muon_shape_t* shapes, int n, muon_mode_t mode, Plan* P) {
     const GroupPlan& gp = P->groups[P->mat_group[i]];
     const int nt = (gp.mp / kEwTileR) * (gp.np / kEwTileC);
     P->ew_ntiles[i] = nt;
-    P->ew_nclusters[i] = (nt + kEwCluster - 1) / kEwCluster;
+    constexpr int per_cluster = kEwCluster * kEwTilesPerCta;
+    P->ew_nclusters[i] = (nt + per_cluster - 1) / per_cluster;
     P->ew_part_begin[i] = parts;
     parts += P->ew_nclusters[i];
   }
@@ -214,6 +216,7 @@ struct muon_ctx {
   float* d_scal = nullptr;
   float* d_partials = nullptr;
   float* d_norms = nullptr;   // ||U_i||_F in caller order
+  bool fuse_shapes_ok = false;  // every group's real dimensions are multiples of 32, n <= kTcMaxFused
   // launch parameter blocks (tens of KB), reused by every call on this handle
   EwParams ew;
   WrParams wr;
@@ -299,9 +302,25 @@ cudaError_t enqueue_front(muon_ctx* h, const void* const* src, void* const* mom,
   return cudaSuccess;
 }
 
-cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, int* launches) {
+// The parameter write can ride on the last Update launch when the parameters are bf16,
+// every real dimension is a multiple of 32 (epilogue chunks are all real or all padding),
+// the pointers fit the launch parameters and every destination is 16-byte aligned.
+bool write_fusable(const muon_ctx* h, void* const* dst, int k) {
+  if (h->mode != MUON_MODE_FAST || h->dtype != MUON_BF16 || k < 1 || !h->fuse_shapes_ok) return false;
+  for (int i = 0; i < h->n; ++i)
+    if ((reinterpret_cast<uintptr_t>(dst[i]) & 15u) != 0) return false;
+  return true;
+}
+
+// k Newton-Schulz iterations.  When *fused comes back true, the last Update has also
+// written dst (the parameter update, or O itself when store_only) and the separate
+// write kernel must not run.
+cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, int* launches, void* const* dst,
+                       bool store_only, bool* fused) {
   const Plan& P = h->plan;
   const int k = hp->ns_steps;
+  const bool fuse = write_fusable(h, dst, k);
+  *fused = fuse;
   for (int t = 1; t <= k; ++t) {
     const int cur = (t - 1) & 1, nxt = t & 1;
     if (h->mode == MUON_MODE_FAST) {
@@ -319,8 +338,23 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
           prm.status = h->d_status;
           prm.timeout_ns = kTimeoutNs;
           if (kind == kGram) { prm.c_acc = 1.0f; prm.c_aux = 0.0f; }
-          if (kind == kPoly) { prm.c_acc = hp->c; prm.c_aux = hp->b; }
-          if (kind == kUpdate) { prm.c_acc = 1.0f; prm.c_aux = hp->a; }
+          // Poly writes B' = a I + b A + c A A (the a X term of the update folded into B'),
+          // so Update is the plain product X' = s * (B' X).
+          if (kind == kPoly) { prm.c_acc = hp->c; prm.c_aux = hp->b; prm.c_diag = hp->a; }
+          if (kind == kUpdate) { prm.c_acc = 1.0f; prm.c_aux = 0.0f; }
+          if (kind == kUpdate && t == k && fuse) {
+            prm.fuse_write = 1;
+            prm.w_decay = store_only ? 0.0f : 1.0f - hp->lr * hp->weight_decay;
+            for (const GroupPlan& gp : P.groups) {
+              for (int sl = 0; sl < gp.cnt; ++sl) {
+                const int i = gp.mats[sl], slot = gp.scal_base + sl;
+                const float r = static_cast<float>(h->shapes[i].rows), c = static_cast<float>(h->shapes[i].cols);
+                prm.wptr[slot] = dst[i];
+                prm.wcoef[slot] = store_only ? 1.0f : -hp->lr * std::sqrt(std::max(1.0f, r / c));
+                prm.wtrans[slot] = h->shapes[i].rows > h->shapes[i].cols ? 1 : 0;
+              }
+            }
+          }
           int tiles = 0;
           for (int gi = 0; gi < ng; ++gi) {
             const GroupPlan& gp = P.groups[g0 + gi];
@@ -340,12 +374,14 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.kblocks = gp.np / kTcBK;
               G.tdim = T;
               G.out_ld = gp.mp;
+              G.m_real = gp.m;
             } else if (kind == kPoly) {
               G.tm_a = gp.tm_a;
               G.tm_b = gp.tm_a;
               G.out = h->ws + gp.off_b;
               G.aux = h->ws + gp.off_a;
               G.tiles_per_mat = T * (T + 1) / 2;
+              G.m_real = gp.m;
               G.kblocks = gp.mp / kTcBK;
               G.tdim = T;
               G.out_ld = gp.mp;
@@ -353,11 +389,13 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_a = gp.tm_b;
               G.tm_b = gp.tm_x[cur];
               G.out = h->ws + gp.off_x[nxt];
-              G.aux = h->ws + gp.off_x[cur];
+              G.aux = nullptr;
               G.tiles_per_mat = (gp.mp / 256) * (gp.np / 256);  // 256 x 256 pair tiles
               G.kblocks = gp.mp / kTcBK;
               G.tdim = gp.np / 256;
               G.out_ld = gp.np;
+              G.m_real = gp.m;
+              G.n_real = gp.n;
             }
             tiles += G.tiles_per_mat * gp.cnt;
           }
@@ -393,13 +431,14 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
             s.lda = gp.mp; s.ldb = gp.mp; s.ldc = gp.mp;
             s.sa = as; s.sb = as; s.sc = as;
             s.b_trans = 0; s.c_acc = hp->c; s.c_aux = hp->b;
+            s.c_diag = hp->a; s.diag_n = gp.m;  // B' = a I + b A + c A A
             s.scal_mode = 0;
           } else {
-            s.a = B; s.b = x; s.c = xn; s.aux = x;
+            s.a = B; s.b = x; s.c = xn; s.aux = nullptr;
             s.M = gp.mp; s.N = gp.np; s.K = gp.mp;
             s.lda = gp.mp; s.ldb = gp.np; s.ldc = gp.np;
             s.sa = as; s.sb = xs; s.sc = xs;
-            s.b_trans = 0; s.c_acc = 1.0f; s.c_aux = hp->a;
+            s.b_trans = 0; s.c_acc = 1.0f; s.c_aux = 0.0f;
             s.scal_mode = (t == 1) ? 2 : 0;
           }
           cudaError_t e = launch_sgemm(s, st);
@@ -464,7 +503,8 @@ int launches_for(const muon_ctx* h, int k) {
   const int chunks = (h->n + kEwMatsPerLaunch - 1) / kEwMatsPerLaunch;
   const int ng = static_cast<int>(h->plan.groups.size());
   const int per_stage = (h->mode == MUON_MODE_FAST) ? (ng + kTcMaxGroups - 1) / kTcMaxGroups : ng;
-  return chunks + 3 * k * per_stage + chunks;
+  const bool fused = h->mode == MUON_MODE_FAST && h->dtype == MUON_BF16 && k >= 1 && h->fuse_shapes_ok;
+  return chunks + 3 * k * per_stage + (fused ? 0 : chunks);
 }
 
 }  // namespace
@@ -521,6 +561,9 @@ muon_status_t muon_create(muon_handle_t* handle, const muon_shape_t* shapes, int
   h->n = n;
   h->shapes.assign(shapes, shapes + n);
   make_plan(shapes, n, mode, &h->plan);
+  h->fuse_shapes_ok = n <= kTcMaxFused;
+  for (const GroupPlan& gp : h->plan.groups)
+    if (gp.m % 32 != 0 || gp.n % 32 != 0) h->fuse_shapes_ok = false;
   if (workspace == nullptr || ws_bytes < h->plan.total || (reinterpret_cast<uintptr_t>(workspace) & 1023u) != 0) {
     delete h;
     return MUON_ERR_WORKSPACE;
@@ -566,9 +609,10 @@ muon_status_t muon_step(muon_handle_t h, void* const* W, const void* const* G, v
     if (W[i] == nullptr || G[i] == nullptr || M[i] == nullptr) return MUON_ERR_INVALID_ARG;
   DeviceGuard guard(h->device);
   int launches = 0;
+  bool fused = false;
   cudaError_t e = enqueue_front(h, G, M, hp, stream, &launches);
-  if (e == cudaSuccess) e = enqueue_ns(h, hp, stream, &launches);
-  if (e == cudaSuccess) e = enqueue_back(h, W, hp, false, stream, &launches);
+  if (e == cudaSuccess) e = enqueue_ns(h, hp, stream, &launches, W, false, &fused);
+  if (e == cudaSuccess && !fused) e = enqueue_back(h, W, hp, false, stream, &launches);
   trace_call_end(h);
   return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
@@ -586,8 +630,9 @@ muon_status_t muon_orthogonalize(muon_handle_t h, const void* const* X, void* co
   q.weight_decay = 0.0f;
   int launches = 0;
   cudaError_t e = enqueue_front(h, X, nullptr, &q, stream, &launches);
-  if (e == cudaSuccess) e = enqueue_ns(h, &q, stream, &launches);
-  if (e == cudaSuccess) e = enqueue_back(h, O, &q, true, stream, &launches);
+  bool fused = false;
+  if (e == cudaSuccess) e = enqueue_ns(h, &q, stream, &launches, O, true, &fused);
+  if (e == cudaSuccess && !fused) e = enqueue_back(h, O, &q, true, stream, &launches);
   trace_call_end(h);
   return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }

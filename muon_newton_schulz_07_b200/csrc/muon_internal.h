@@ -23,6 +23,7 @@ constexpr int kEwTileR = 64;
 constexpr int kEwTileC = 128;
 constexpr int kEwThreads = 256;
 constexpr int kEwCluster = 8;       // CTAs per cluster in the momentum/norm kernel
+constexpr int kEwTilesPerCta = 2;   // tiles per CTA in the momentum/norm kernel
 constexpr int kEwMatsPerLaunch = 192;
 
 enum Dtype : int { kBF16 = 0, kF32 = 1 };
@@ -36,7 +37,7 @@ struct EwMat {
   int trans;         // rows > cols: X = U^T
   int tile_begin;    // first CTA (cluster aligned) of this matrix in the launch
   int tiles_c;       // X tiles along np
-  int ntiles;        // X tiles of the padded matrix (mp/64 * np/128)
+  int ntiles;        // X tiles of the padded matrix (mp/64 * np/128), kEwTilesPerCta per CTA
   int scal_idx;      // slot of this matrix in the scalar / counter tables
   int caller_idx;    // position in the caller's matrix list
   int part_begin;    // first per-cluster partial slot
@@ -103,8 +104,14 @@ struct alignas(64) TcGroup {
   int scal_base;
   int tdim;             // Gram/Poly: mp/256 (triangle side); Update: np/256
   int out_ld;
-  int pad_[3];
+  int m_real;           // real (unpadded) rows: Poly adds its diagonal term only there
+  int n_real;           // real (unpadded) columns of X
+  int pad_;
 };
+
+// Largest number of matrices whose parameter write can be fused into the last
+// Update launch (their pointers travel in the kernel parameters).
+constexpr int kTcMaxFused = 1024;
 
 struct TcParams {
   TcGroup g[kTcMaxGroups];
@@ -112,10 +119,20 @@ struct TcParams {
   int total_tiles;
   int kind;
   int use_scal;          // first iteration: fold the normalisation in
-  float c_acc, c_aux;    // out = s * (c_acc * acc + c_aux * aux)
+  float c_acc, c_aux;    // out = s * (c_acc * acc + c_aux * aux) (+ c_diag on the real diagonal)
+  float c_diag;
   const float* scal;
   unsigned int* status;
   unsigned long long timeout_ns;
+  // Fused parameter write (last Update only).  Instead of storing X_k, the epilogue
+  // writes W = w_decay * W + wcoef[slot] * X_k into the caller's bf16 matrix of each
+  // slot (the scalar-table index), transposed back when wtrans[slot] is set.  With
+  // w_decay == 0 it stores wcoef * X_k without reading W (the orthogonaliser output).
+  int fuse_write;
+  float w_decay;
+  void* wptr[kTcMaxFused];
+  float wcoef[kTcMaxFused];
+  unsigned char wtrans[kTcMaxFused];
 };
 
 size_t tc_smem_bytes();
@@ -131,6 +148,7 @@ struct SgParams {
   int b_trans;            // 1: second operand is b^T (b row-major N x K)
   float c_acc, c_aux;
   const float* scal; int scal_base; int scal_mode;  // 0: none, 1: alpha^2, 2: alpha
+  float c_diag; int diag_n;  // add c_diag to C[i][i] for i < diag_n
 };
 cudaError_t launch_sgemm(const SgParams& p, cudaStream_t s);
 

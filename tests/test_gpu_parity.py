@@ -154,7 +154,8 @@ def test_intermediates_symmetric_and_padded():
         U = to_f64(x)
         Xn = O.frobenius_normalize(U.T if U.shape[0] > U.shape[1] else U, 1e-7)
         A_ref = Xn @ Xn.T
-        B_ref = b * A_ref + c * (A_ref @ A_ref)
+        # the polynomial matrix carries the a X term of the update: B' = a I + b A + c A A
+        B_ref = a * np.eye(m) + b * A_ref + c * (A_ref @ A_ref)
         assert rel_fro(A[:m, :m], A_ref) < 2 * 2.0 ** -8
         assert rel_fro(Bm[:m, :m], B_ref) < 4 * 2.0 ** -8
 
