@@ -21,9 +21,11 @@
 // 128 x 256 tile needs.  The even CTA issues the MMAs; its commits are
 // multicast to the barriers of both CTAs.
 //
-// Gram and Poly outputs are symmetric: only 256 x 256 tiles on or above the
-// diagonal are computed; every element on or above the diagonal is stored at
-// (r, c) and mirrored to (c, r), so the result is exactly symmetric.
+// Gram and Poly outputs are symmetric: only the 256 x 256 blocks on or above the
+// diagonal are computed and stored (diagonal blocks in full).  Whoever needs a
+// block below the diagonal (Poly reading A, Update reading B') TMA-loads the
+// stored block above it and feeds it to the tensor core as an MN-major operand,
+// so the lower halves of A and B' are never written or read.
 //
 // Roles in each CTA (192 threads, one CTA per SM, persistent over a static
 // round-robin list of pair tiles):
@@ -36,12 +38,14 @@
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, the fp32 combination
 //               (Poly: c A A + b A + a I), bf16 cast, stores staged through
 //               shared memory so every global access is a 64-byte row run
-//               (plus the mirrored store for Gram/Poly).  In the last Update
+//               (upper blocks only for Gram/Poly).  In the last Update
 //               the epilogue writes the parameters directly:
 //               W = (1 - lr wd) W - lr sqrt(max(1, r/c)) X_k from the unrounded
 //               fp32 X_k, transposed back for tall matrices.
-// Operand B of Update is X itself in its row-major layout, i.e. MN-major; the
-// other operands are K-major.  All waits are bounded (see muon_device.cuh).
+// Operand B of Update is X itself in its row-major layout, i.e. MN-major, and so
+// is every transposed block of A or B'; the other operands are K-major.  The
+// instruction descriptor's major bits are set per k slice.  All waits are
+// bounded (see muon_device.cuh).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -71,6 +75,7 @@ struct Tile {
   int g, mat, row0, col0;
 };
 
+template <int KIND>
 __device__ __forceinline__ Tile decode_tile(const TcParams& p, int t) {
   int g = 0;
   while (g + 1 < p.ngroups && p.g[g + 1].tile_begin <= t) ++g;
@@ -81,7 +86,7 @@ __device__ __forceinline__ Tile decode_tile(const TcParams& p, int t) {
   Tile ti;
   ti.g = g;
   ti.mat = mat;
-  if (p.kind == kUpdate) {
+  if (KIND == kUpdate) {
     const int tm = r / G.tdim;
     ti.row0 = tm * TILE;
     ti.col0 = (r - tm * G.tdim) * TILE;
@@ -115,6 +120,7 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
   return q;
 }
 
+template <int KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     ns_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -168,10 +174,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       const int half = static_cast<int>(rank) * (BN / 2);
+      constexpr bool sym_a = KIND != kGram;         // A (Poly) and B' (Update) are stored as upper blocks
+      constexpr bool sym_b = KIND == kPoly;
+      constexpr bool ta_update_b = KIND == kUpdate;  // X is always read MN-major by Update
       for (int t = cl; t < p.total_tiles; t += ncl) {
-        const Tile ti = decode_tile(p, t);
+        const Tile ti = decode_tile<KIND>(p, t);
         const TcGroup& G = p.g[ti.g];
         const int arow = ti.row0 + static_cast<int>(rank) * BM;
+        const int ia = ti.row0 / TILE, jb = ti.col0 / TILE;
         bool ok = true;
         for (int kb = 0; kb < G.kblocks; ++kb) {
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, p.status)) {
@@ -182,9 +192,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
           const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + A_STAGE;
           const int k0 = kb * BK;
-          tma_load_3d_pair(sa, &G.tm_a, fb, k0, arow, ti.mat);
-          tma_load_3d_pair(sa + BOX_BYTES, &G.tm_a, fb, k0, arow + 64, ti.mat);
-          if (p.kind != kUpdate) {
+          // Blocks of A / B' below the diagonal are not stored: load the transposed block
+          // above it instead (the MMA reads it MN-major).
+          const bool ta = sym_a && k0 / TILE < ia;
+          const bool tb = sym_b && k0 / TILE < jb;
+          const bool mnb = ta_update_b || tb;
+          if (!ta) {
+            tma_load_3d_pair(sa, &G.tm_a, fb, k0, arow, ti.mat);
+            tma_load_3d_pair(sa + BOX_BYTES, &G.tm_a, fb, k0, arow + 64, ti.mat);
+          } else {
+            tma_load_3d_pair(sa, &G.tm_a, fb, arow, k0, ti.mat);
+            tma_load_3d_pair(sa + BOX_BYTES, &G.tm_a, fb, arow + 64, k0, ti.mat);
+          }
+          if (!mnb) {
             tma_load_3d_pair(sb, &G.tm_b, fb, k0, ti.col0 + half, ti.mat);
             tma_load_3d_pair(sb + BOX_BYTES, &G.tm_b, fb, k0, ti.col0 + half + 64, ti.mat);
           } else {
@@ -212,18 +232,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------- MMA issuer (even CTA)
-      const uint32_t idesc = idesc_bf16_f32(2 * BM, BN, 0, p.kind == kUpdate ? 1 : 0);
+      constexpr bool sym_a = KIND != kGram;
+      constexpr bool sym_b = KIND == kPoly;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = cl; t < p.total_tiles && ok; t += ncl) {
-        const Tile ti = decode_tile(p, t);
+        const Tile ti = decode_tile<KIND>(p, t);
         const TcGroup& G = p.g[ti.g];
         if (!mbar_wait_bounded(acce_bar(acc), acc_phase ^ 1u, tmo, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const int ia = ti.row0 / TILE, jb = ti.col0 / TILE;
         for (int kb = 0; kb < G.kblocks; ++kb) {
           if (!mbar_wait_bounded(full_bar(stage), phase, tmo, abort_flag, p.status)) {
             ok = false;
@@ -231,13 +253,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + A_STAGE;
+          const int kk = kb * BK / TILE;
+          const bool mna = sym_a && kk < ia;                        // transposed block of A / B'
+          const bool mnb = (KIND == kUpdate) || (sym_b && kk < jb);
+          const uint32_t idesc = idesc_bf16_f32(2 * BM, BN, mna ? 1 : 0, mnb ? 1 : 0);
+          // K-major: 16 k per step = 32 bytes along the swizzled row; MN-major: 16 k rows
+          // = 2 KB, with the two 64-wide M/N chunks 8 KB apart.  The start address sits
+          // in the low bits of the descriptor (16-byte units), so a step is a plain add.
+          const uint64_t adesc0 = mna ? smem_desc_sw128(sa, 8192, 1024) : smem_desc_sw128(sa, 16, 1024);
+          const uint64_t bdesc0 = mnb ? smem_desc_sw128(sb, 8192, 1024) : smem_desc_sw128(sb, 16, 1024);
+          const uint64_t astep = mna ? (2048u >> 4) : (32u >> 4);
+          const uint64_t bstep = mnb ? (2048u >> 4) : (32u >> 4);
 #pragma unroll
-          for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t adesc = smem_desc_sw128(sa + 32u * j, 16, 1024);
-            const uint64_t bdesc = (p.kind == kUpdate) ? smem_desc_sw128(sb + 2048u * j, 8192, 1024)
-                                                       : smem_desc_sw128(sb + 32u * j, 16, 1024);
-            tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | j) != 0 ? 1u : 0u);
-          }
+          for (int j = 0; j < BK / 16; ++j)
+            tc_mma_bf16_pair(d_tmem, adesc0 + astep * j, bdesc0 + bstep * j, idesc, (kb | j) != 0 ? 1u : 0u);
           tc_commit_pair_mc(empty_bar(stage), 0x3);  // frees the stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
@@ -260,11 +289,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + EPI_OFFSET + (warp - 2) * EPI_WARP_BYTES);
     __nv_bfloat16* stg_aux = stg + 32 * EPI_PITCH;
     const int sub_r = lane >> 2, sub_c = (lane & 3) * 8;
-    const bool symmetric = (p.kind != kUpdate);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = cl; t < p.total_tiles; t += ncl) {
-      const Tile ti = decode_tile(p, t);
+      const Tile ti = decode_tile<KIND>(p, t);
       const TcGroup& G = p.g[ti.g];
       const int ld = G.out_ld;
       const size_t mat_off = static_cast<size_t>(ti.mat) * G.mp * ld;
@@ -272,105 +300,106 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       const __nv_bfloat16* aux = G.aux ? static_cast<const __nv_bfloat16*>(G.aux) + mat_off : nullptr;
       const int gr0 = ti.row0 + static_cast<int>(rank) * BM + quad * 32;  // first row of this warp
       const int gr = gr0 + lane;
-      // The auxiliary input does not depend on the accumulator: fetch its first chunk
-      // (the first one at or above the diagonal) before waiting, and every later chunk
-      // one step ahead, so its latency hides behind the accumulator drain.
-      uint4 pf[4];
-      auto aux_load = [&](int c, uint4 (&dst)[4]) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          dst[q] = __ldg(reinterpret_cast<const uint4*>(aux + static_cast<size_t>(gr0 + q * 8 + sub_r) * ld +
-                                                        ti.col0 + c * 32 + sub_c));
-      };
-      if (aux != nullptr) {
-        int c0 = 0;
-        while (symmetric && c0 < BN / 32 - 1 && ti.col0 + c0 * 32 + 32 <= gr0) ++c0;
-        aux_load(c0, pf);
+      // Fused parameter write (last Update): the caller's matrix of this tile.
+      const bool fw = p.fuse_write != 0;
+      __nv_bfloat16* W = nullptr;
+      float cw = 0.0f;
+      bool tr = false;
+      int ldw = 0;
+      if (fw) {
+        const int slot = G.scal_base + ti.mat;
+        W = static_cast<__nv_bfloat16*>(p.wptr[slot]);
+        cw = p.wcoef[slot];
+        tr = p.wtrans[slot] != 0;
+        ldw = tr ? G.m_real : G.n_real;
       }
+      const bool wread = fw && p.w_decay != 0.0f && gr0 < G.m_real;
+      // element (row rr, 8 columns from sub_c) of the chunk at column gc in W's own layout
+      auto woff = [&](int gc, int rr) -> size_t {
+        return tr ? static_cast<size_t>(gc + rr) * ldw + gr0 + sub_c : static_cast<size_t>(gr0 + rr) * ldw + gc + sub_c;
+      };
+      // The auxiliary input (A for Poly, W for the fused Update) does not depend on the
+      // accumulator: fetch its first chunk (the first at or above the diagonal) before
+      // waiting, and every later chunk one step ahead, so its latency hides behind the
+      // accumulator drain.
+      uint4 pf[4];
+      auto pre_load = [&](int c, uint4 (&dst)[4]) {
+        const int gc = ti.col0 + c * 32;
+        if (aux != nullptr) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = __ldg(reinterpret_cast<const uint4*>(aux + static_cast<size_t>(gr0 + q * 8 + sub_r) * ld + gc + sub_c));
+        } else if (wread && gc < G.n_real) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = __ldcs(reinterpret_cast<const uint4*>(W + woff(gc, q * 8 + sub_r)));
+        }
+      };
+      const bool has_pre = aux != nullptr || wread;
+      if (has_pre) pre_load(0, pf);
       if (!mbar_wait_bounded(accf_bar(acc), acc_phase, tmo, abort_flag, p.status)) break;
       tc_fence_after();
       float s = 1.0f;
       if (p.use_scal) {
         const float al = p.scal[2 * (G.scal_base + ti.mat) + 1];
-        s = (p.kind == kGram) ? al * al : al;
+        s = (KIND == kGram) ? al * al : al;
       }
-      const float cdiag = (p.kind == kPoly && gr < G.m_real) ? p.c_diag : 0.0f;
+      const float cdiag = (KIND == kPoly && gr < G.m_real) ? p.c_diag : 0.0f;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const uint32_t acce_leader = map_to_rank(acce_bar(acc), 0);
 #pragma unroll 1
       for (int ch = 0; ch < BN / 32; ++ch) {
         const int gc0 = ti.col0 + ch * 32;
-        // Chunks of Gram/Poly tiles lie fully above the diagonal, on it, or fully below it
-        // (rows and columns are both multiples of 32); the ones below are mirrored from
-        // elsewhere.  The last chunk of a tile is never below the diagonal.
-        const bool below = symmetric && gc0 + 32 <= gr0;
-        const bool diag = symmetric && gc0 == gr0;
         float v[32];
-        if (!below) {
-          __syncwarp();
-          tmem_ld_32cols(taddr + ch * 32, v);
-        }
+        __syncwarp();
+        tmem_ld_32cols(taddr + ch * 32, v);
         if (ch == BN / 32 - 1) {
           // all of this accumulator has been read: hand it back to the MMA issuer
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_remote(acce_leader);
         }
-        if (below) continue;
-        if (p.fuse_write) {
+        uint4 nx[4];
+        if (has_pre && ch + 1 < BN / 32) pre_load(ch + 1, nx);
+        if (fw) {
           // Last Update: write the parameters instead of X_k.  Chunks in the zero padding
           // of the workspace have no parameters (real dimensions are multiples of 32).
-          if (gr0 >= G.m_real || gc0 >= G.n_real) continue;
-          const int slot = G.scal_base + ti.mat;
-          __nv_bfloat16* W = static_cast<__nv_bfloat16*>(p.wptr[slot]);
-          const float cw = p.wcoef[slot];
-          const bool tr = p.wtrans[slot] != 0;
-          const int ldw = tr ? G.m_real : G.n_real;
-          // element (row rr, 8 columns from sub_c) of this chunk in W's own layout
-          auto woff = [&](int rr) -> size_t {
-            return tr ? static_cast<size_t>(gc0 + rr) * ldw + gr0 + sub_c
-                      : static_cast<size_t>(gr0 + rr) * ldw + gc0 + sub_c;
-          };
-          uint4 wv[4];
-          if (p.w_decay != 0.0f) {
+          if (gr0 < G.m_real && gc0 < G.n_real) {
+            // stage s * acc in fp32 (row-major, or transposed for tall parameters)
+            float* st32 = reinterpret_cast<float*>(stg);
+            if (!tr) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) wv[q] = __ldcs(reinterpret_cast<const uint4*>(W + woff(q * 8 + sub_r)));
-          }
-          // stage s * acc in fp32 (row-major, or transposed for tall parameters)
-          float* st32 = reinterpret_cast<float*>(stg);
-          if (!tr) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(st32 + lane * F32_PITCH + i) =
-                  make_float4(s * v[i], s * v[i + 1], s * v[i + 2], s * v[i + 3]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) st32[i * F32_PITCH + lane] = s * v[i];
-          }
-          __syncwarp();
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int rr = q * 8 + sub_r;
-            const float4 o0 = *reinterpret_cast<const float4*>(st32 + rr * F32_PITCH + sub_c);
-            const float4 o1 = *reinterpret_cast<const float4*>(st32 + rr * F32_PITCH + sub_c + 4);
-            float r8[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-            if (p.w_decay != 0.0f) {
-              float w8[8];
-              unpack8(wv[q], w8);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) r8[i] = fmaf(p.w_decay, w8[i], cw * r8[i]);
+              for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(st32 + lane * F32_PITCH + i) =
+                    make_float4(s * v[i], s * v[i + 1], s * v[i + 2], s * v[i + 3]);
             } else {
 #pragma unroll
-              for (int i = 0; i < 8; ++i) r8[i] = cw * r8[i];
+              for (int i = 0; i < 32; ++i) st32[i * F32_PITCH + lane] = s * v[i];
             }
-            __stcs(reinterpret_cast<uint4*>(W + woff(rr)), pack8(r8));
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int rr = q * 8 + sub_r;
+              const float4 o0 = *reinterpret_cast<const float4*>(st32 + rr * F32_PITCH + sub_c);
+              const float4 o1 = *reinterpret_cast<const float4*>(st32 + rr * F32_PITCH + sub_c + 4);
+              float r8[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+              if (wread) {
+                float w8[8];
+                unpack8(pf[q], w8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) r8[i] = fmaf(p.w_decay, w8[i], cw * r8[i]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) r8[i] = cw * r8[i];
+              }
+              __stcs(reinterpret_cast<uint4*>(W + woff(gc0, rr)), pack8(r8));
+            }
+            __syncwarp();
           }
-          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) pf[q] = nx[q];
           continue;
         }
         if (aux != nullptr) {
-          uint4 nx[4];
-          if (ch + 1 < BN / 32) aux_load(ch + 1, nx);  // a chunk after a non-skipped one is never skipped
 #pragma unroll
           for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(stg_aux + (q * 8 + sub_r) * EPI_PITCH + sub_c) = pf[q];
 #pragma unroll
@@ -387,19 +416,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = s * p.c_acc * v[i];
         }
-        if (diag) {
+        if (gc0 == gr0) {
+          // the chunk on the diagonal: Poly adds a on the real diagonal (B' = a I + ...)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (gc0 + i == gr) v[i] += cdiag;
-          // on-diagonal chunk: element-wise, keeping (r, c) with c >= r and mirroring c > r
-          __nv_bfloat16* orow = out + static_cast<size_t>(gr) * ld + gc0;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (gc0 + i >= gr) orow[i] = __float2bfloat16_rn(v[i]);
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (gc0 + i > gr) out[static_cast<size_t>(gc0 + i) * ld + gr] = __float2bfloat16_rn(v[i]);
-          continue;
         }
         // direct store: row-major staging, then 64-byte row runs
 #pragma unroll
@@ -410,19 +431,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           const int rr = q * 8 + sub_r;
           *reinterpret_cast<uint4*>(out + static_cast<size_t>(gr0 + rr) * ld + gc0 + sub_c) =
               *reinterpret_cast<const uint4*>(stg + rr * EPI_PITCH + sub_c);
-        }
-        if (symmetric) {
-          // mirrored store: transposed staging, then 64-byte runs of the mirrored rows
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) stg[i * EPI_PITCH + lane] = __float2bfloat16_rn(v[i]);
-          __syncwarp();
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int cc = q * 8 + sub_r;
-            *reinterpret_cast<uint4*>(out + static_cast<size_t>(gc0 + cc) * ld + gr0 + sub_c) =
-                *reinterpret_cast<const uint4*>(stg + cc * EPI_PITCH + sub_c);
-          }
         }
       }
       acc ^= 1;
@@ -441,23 +449,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   }
 }
 
+template <int KIND>
+cudaError_t launch_kind(const TcParams& p, int grid, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  ns_gemm_tc_kernel<KIND><<<grid, kTcThreads, SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t tc_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(SMEM_BYTES));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   // one CTA pair per TPC, at most one pair per tile
-  const int pairs = std::min(num_sms / 2, p.total_tiles);
-  ns_gemm_tc_kernel<<<2 * pairs, kTcThreads, SMEM_BYTES, s>>>(p);
-  return cudaGetLastError();
+  const int grid = 2 * std::min(num_sms / 2, p.total_tiles);
+  if (p.kind == kGram) return launch_kind<kGram>(p, grid, s);
+  if (p.kind == kPoly) return launch_kind<kPoly>(p, grid, s);
+  return launch_kind<kUpdate>(p, grid, s);
 }
 
 }  // namespace muon
