@@ -71,6 +71,25 @@ def bytes_by_kind(shapes, elem=2):
     return {"momentum_norm": 4 * elem * n, "write": 3 * elem * n}
 
 
+def measured_traffic(kind, workload):
+    """DRAM bytes (read + write) per launch of the dominant kernel from the committed ncu capture,
+    scaled to the workload; None unless the capture matches this kernel source and workload."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", f"traffic_{kind}_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != rec["source_sha256_16"]:
+            return None  # the kernel changed since the counters were taken
+    scale = rec["scale_to_workload"].get(workload)
+    if scale is None:
+        return None
+    return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * scale
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -355,7 +374,7 @@ def run_muon(args, rank, world, local_rank):
         ach = per_launch_units[dominant] / (kern[dominant]["ms_per_launch"] * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                "traffic": None, "kernel": f"ns_gemm_tc_kernel ({dominant})",
+                "traffic": measured_traffic(dominant, wl.name), "kernel": f"ns_gemm_tc_kernel ({dominant})",
                 "peak_source": f"{peak_src} bf16_tflops_sustained"}
     else:
         ach = per_launch_units[dominant] / (kern[dominant]["ms_per_launch"] * 1e-3) / 1e9
