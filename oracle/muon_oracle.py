@@ -49,6 +49,8 @@ Parity pins (tests/test_oracle.py, all CPU):
     transpose symmetry, scale invariance, orthogonal equivariance, fixed points
     of orthonormal inputs; a hand-derived 2x2 diagonal example.
   * the matmul primitive against a brute-force triple loop.
+  * adamw_step: a hand-derived first step, the closed form for a constant gradient
+    (bias-corrected moments equal g and g^2 at every step), the beta = 0 special case.
 No function here is unpinned.
 """
 from __future__ import annotations
@@ -174,6 +176,33 @@ def muon_step_set(Ws, Gs, Ms, hp: Hyper):
     """The step over a parameter set: each matrix independently, in order."""
     out = [muon_step(W, G, M, hp) for W, G, M in zip(Ws, Gs, Ms)]
     return [o[0] for o in out], [o[1] for o in out], [o[2] for o in out]
+
+
+# ---------------------------------------------------------------------------
+# AdamW for the parameters that are not matrices.
+# ---------------------------------------------------------------------------
+
+def adamw_step(p, g, m, v, step: int, lr: float, beta1: float, beta2: float, eps: float,
+               weight_decay: float):
+    """One AdamW step (returns p1, m1, v1 as float64).
+
+    The hybrid recipe hands every parameter that is not a 2-D matrix to AdamW
+    ("开发者千美元训3.8B模型 击败GPT-2", aiproducthub, 影响 paragraph).  The pages
+    give no formula; this is the plainest reading, the decoupled-weight-decay Adam
+    with bias correction, in its usual order:
+      m1 = beta1 m + (1 - beta1) g;  v1 = beta2 v + (1 - beta2) g^2
+      mh = m1 / (1 - beta1^t);       vh = v1 / (1 - beta2^t)      (t = step >= 1)
+      p1 = (1 - lr wd) p - lr mh / (sqrt(vh) + eps)
+    """
+    p, g, m, v = _f64(p), _f64(g), _f64(m), _f64(v)
+    if step < 1:
+        raise ValueError("step counts from 1")
+    m1 = beta1 * m + (1.0 - beta1) * g
+    v1 = beta2 * v + (1.0 - beta2) * g * g
+    mh = m1 / (1.0 - beta1 ** step)
+    vh = v1 / (1.0 - beta2 ** step)
+    p1 = (1.0 - lr * weight_decay) * p - lr * mh / (np.sqrt(vh) + eps)
+    return p1, m1, v1
 
 
 # ---------------------------------------------------------------------------

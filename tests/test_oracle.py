@@ -282,3 +282,50 @@ def test_pins_catch_planted_mistakes(mutant, monkeypatch):
     bad = mo.newton_schulz(X, 3)
     assert rel(good, O.spectral_newton_schulz(X, 3)) < 1e-12
     assert rel(bad, O.spectral_newton_schulz(X, 3)) > 1e-3
+
+
+# ---------------------------------------------------------------- AdamW (the non-matrix half)
+
+def test_adamw_first_step_worked_example():
+    # t = 1, m = v = 0: m1 = 0.1 g, v1 = 0.001 g^2, corrected to g and g^2, so with eps = 0
+    # the step is lr * sign(g); p = 1, g = 2, lr = 0.1 -> 0.9; with wd = 0.5 -> 0.95 - 0.1
+    p1, m1, v1 = O.adamw_step(np.array([1.0]), np.array([2.0]), np.zeros(1), np.zeros(1), 1,
+                              lr=0.1, beta1=0.9, beta2=0.999, eps=0.0, weight_decay=0.0)
+    assert abs(m1[0] - 0.2) < 1e-15 and abs(v1[0] - 0.004) < 1e-15
+    assert abs(p1[0] - 0.9) < 1e-14
+    p1, _, _ = O.adamw_step(np.array([1.0]), np.array([2.0]), np.zeros(1), np.zeros(1), 1,
+                            lr=0.1, beta1=0.9, beta2=0.999, eps=0.0, weight_decay=0.5)
+    assert abs(p1[0] - 0.85) < 1e-14
+
+
+def test_adamw_constant_gradient_closed_form():
+    # with a constant gradient the bias-corrected moments are exactly g and g^2 at every step,
+    # so T steps move p by T * lr * g / (|g| + eps)
+    rng = np.random.default_rng(20)
+    g = rng.standard_normal(50)
+    p0 = rng.standard_normal(50)
+    p, m, v = p0.copy(), np.zeros(50), np.zeros(50)
+    for t in range(1, 8):
+        p, m, v = O.adamw_step(p, g, m, v, t, lr=1e-2, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.0)
+    assert np.max(np.abs(p - (p0 - 7 * 1e-2 * g / (np.abs(g) + 1e-8)))) < 1e-12
+
+
+def test_adamw_zero_betas():
+    # beta1 = beta2 = 0: no memory, the step is lr * g / (|g| + eps) whatever m and v held
+    rng = np.random.default_rng(21)
+    p, g, m, v = (rng.standard_normal(30) for _ in range(4))
+    v = np.abs(v)
+    p1, m1, v1 = O.adamw_step(p, g, m, v, 3, lr=0.05, beta1=0.0, beta2=0.0, eps=1e-6, weight_decay=0.0)
+    assert np.array_equal(m1, g) and np.array_equal(v1, g * g)
+    assert np.max(np.abs(p1 - (p - 0.05 * g / (np.abs(g) + 1e-6)))) < 1e-15
+
+
+def test_adamw_pin_catches_missing_bias_correction():
+    rng = np.random.default_rng(22)
+    g = rng.standard_normal(10)
+    m1 = 0.1 * g
+    v1 = 0.05 * g * g
+    wrong = -1e-2 * m1 / (np.sqrt(v1) + 1e-8)  # the step without bias correction
+    right = O.adamw_step(np.zeros(10), g, np.zeros(10), np.zeros(10), 1, lr=1e-2, beta1=0.9, beta2=0.95,
+                         eps=1e-8, weight_decay=0.0)[0]
+    assert np.max(np.abs(right - wrong)) > 1e-3
