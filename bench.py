@@ -37,10 +37,14 @@ def parse():
     ap.add_argument("--impl", choices=["muon", "reference"], default="muon")
     ap.add_argument("--workload", default="d24", choices=["gpt2s", "d24", "l38b", "stress"])
     ap.add_argument("--ns-steps", type=int, default=5)
+    ap.add_argument("--mode", choices=["replica", "sharded"], default="replica",
+                    help="replica: every rank steps its own parameter set (weak scaling); sharded: the ranks "
+                         "split one set by matrix and all-gather the parameters (strong scaling)")
     ap.add_argument("--matrices", type=int, default=0,
                     help="use only the first N matrices of the workload (profiling captures of a smaller case)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW leg (non-matrix parameters)")
     ap.add_argument("--reference-budget-s", type=float, default=150.0)
     return ap.parse_args()
 
@@ -293,7 +297,23 @@ def run_muon(args, rank, world, local_rank):
     W = gen(lambda i: I.weight(wl, i))
     M = gen(lambda i: I.momentum(wl, i))
     G_sets = [gen(lambda i, s=s: I.gradient(wl, 1 + s + 1000 * rank, i)) for s in range(2)]
-    op = MuonStep(shapes, dtype=dt, device=dev)
+    sharded = args.mode == "sharded" and world > 1
+    if sharded:
+        # strong scaling: each rank owns a share of the matrices, steps only those and all-gathers W
+        from muon_newton_schulz_07_b200.sharding import ShardedMuon
+
+        probe = ShardedMuon(shapes, rank, world, local_step=lambda *a, **kw: None, ns_steps=k)
+        op = MuonStep([shapes[i] for i in probe.owned], dtype=dt, device=dev)
+        sh = ShardedMuon(shapes, rank, world, local_step=op, ns_steps=k)
+        M_owned = [M[i] for i in sh.owned]
+
+        def step_fn(Gs):
+            sh.step(W, Gs, M_owned, ns_steps=k)
+    else:
+        op = MuonStep(shapes, dtype=dt, device=dev)
+
+        def step_fn(Gs):
+            op(W, Gs, M, ns_steps=k)
     launches = op.launches_per_step(k)
     stream = torch.cuda.current_stream(dev)
 
@@ -310,7 +330,7 @@ def run_muon(args, rank, world, local_rank):
         return float(t.item())
 
     for i in range(args.warmup):
-        op(W, G_sets[i % 2], M, ns_steps=k)
+        step_fn(G_sets[i % 2])
     sync_all()
     if op.status() != B.MUON_OK:
         raise RuntimeError("device status after warm-up is not OK")
@@ -323,7 +343,7 @@ def run_muon(args, rank, world, local_rank):
     sync_all()
     e0.record(stream)
     for i in range(args.steps):
-        op(W, G_sets[i % 2], M, ns_steps=k)
+        step_fn(G_sets[i % 2])
     e1.record(stream)
     sync_all()
     clk = clocks.stop()
@@ -333,7 +353,7 @@ def run_muon(args, rank, world, local_rank):
     if status != B.MUON_OK:
         raise RuntimeError(f"device status after the timed steps: {B.STATUS.get(status, status)}")
     ms_per_step = max_over_ranks(ms_total / args.steps)
-    value = world * 1000.0 / ms_per_step
+    value = (1 if sharded else world) * 1000.0 / ms_per_step
 
     # ------------------------------------------------------------ end to end (host buffers)
     e2e = None
@@ -349,14 +369,14 @@ def run_muon(args, rank, world, local_rank):
         for i in range(ksteps):
             for d, h in zip(G_dev, G_host[i % 2]):
                 d.copy_(h, non_blocking=True)
-            op(W, G_dev, M, ns_steps=k)
-            op.norms(out=norms_host[i])
+            step_fn(G_dev)
+            op.norms(out=norms_host[i][:len(op.shapes)])
         f1.record(stream)
         sync_all()
         assert np.isfinite(norms_host.numpy()).all()
         e2e_ms = max_over_ranks(f0.elapsed_time(f1) / ksteps)
-        e2e = {"value": world * 1000.0 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": 4 * n, "ms_per_step": e2e_ms, "steps": ksteps,
+        e2e = {"value": (1 if sharded else world) * 1000.0 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": 4 * len(op.shapes), "ms_per_step": e2e_ms, "steps": ksteps,
                "path": "pinned host G -> device copy, MuonStep.__call__ (C ABI muon_step), norms -> pinned host"}
 
     # ------------------------------------------------------------ roofline
@@ -392,6 +412,35 @@ def run_muon(args, rank, world, local_rank):
             kd["gbs"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e9
             kd["frac_of_hbm"] = kd["gbs"] / peaks["hbm_gbs"]
 
+    # ------------------------------------------------------------ AdamW leg (the non-matrix half)
+    adamw = None
+    if not args.no_adamw and wl.name == "d24":
+        from muon_newton_schulz_07_b200.optimizer import adamw_step
+
+        sizes = I.D24_ADAMW_SIZES
+        with ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
+            P = [to_dev(a) for a in ex.map(lambda i: I.adamw_param(0, i, I.TID_W, sizes[i]), range(len(sizes)))]
+            Gd = [to_dev(a) for a in ex.map(lambda i: I.adamw_param(1, i, I.TID_G, sizes[i]), range(len(sizes)))]
+        Ma = [torch.zeros(n, dtype=torch.float32, device=dev) for n in sizes]
+        Va = [torch.zeros(n, dtype=torch.float32, device=dev) for n in sizes]
+        for i in range(args.warmup):
+            adamw_step(P, Gd, Ma, Va, i + 1, lr=3e-3, betas=(0.8, 0.95), eps=1e-10, weight_decay=0.0)
+        sync_all()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(args.steps):
+            adamw_step(P, Gd, Ma, Va, args.warmup + i + 1, lr=3e-3, betas=(0.8, 0.95), eps=1e-10, weight_decay=0.0)
+        a1.record(stream)
+        sync_all()
+        a_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
+        nel = sum(sizes)
+        a_bytes = nel * (2 + 2 + 2 + 8 + 8)  # p read+write, g read, m and v read+write (fp32)
+        a_gbs = a_bytes / (a_ms * 1e-3) / 1e9
+        adamw = {"params": nel, "ms_per_step": a_ms, "gbs": a_gbs, "frac_of_hbm": a_gbs / load_peaks()[0]["hbm_gbs"],
+                 "bytes_per_step": a_bytes, "launches_per_step": 1,
+                 "set": "d24 non-matrix parameters: 14 x 32768x1536 tables + 48 scalars, bf16, fp32 moments"}
+        del P, Gd, Ma, Va
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         step_s, sample = oracle_sample(wl)
@@ -400,10 +449,13 @@ def run_muon(args, rank, world, local_rank):
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "matrices": n, "params": I.param_count(wl), "ns_steps": k,
-                       "groups": op.n_groups, "parallelism": f"replica x{world} (one parameter set per GPU)",
+                       "groups": op.n_groups,
+                       "parallelism": (f"sharded by matrix over {world} ranks + all-gather of W (NCCL)" if sharded
+                                       else f"replica x{world} (one parameter set per GPU)"),
                        "l2": "inputs larger than L2 (W, G, M: %.2f GB per GPU), no flush" %
                              (3 * 2 * I.param_count(wl) / 1e9),
                        "description": wl.description},
@@ -413,6 +465,7 @@ def run_muon(args, rank, world, local_rank):
                    if ns_tflops else None, "ms_per_step": ns_ms, "flops_per_step": ns_flops},
             "kernels": kern,
             "cpu_baseline": cpu,
+            "adamw": adamw,
             "e2e": e2e,
             "gpu_launches": launches * args.steps,
             "clocks": clk,

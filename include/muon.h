@@ -136,6 +136,30 @@ MUON_API muon_status_t muon_orthogonalize(muon_handle_t handle, const void* cons
                                  const muon_hparams_t* hp, cudaStream_t stream);
 
 /*
+ * AdamW for the parameters that are not matrices: the other half of the hybrid
+ * optimizer ("开发者千美元训3.8B模型 击败GPT-2", aiproducthub, 影响 paragraph:
+ * Newton-Schulz orthogonalisation for the matrix parameters, AdamW for the rest).
+ * The pages print no formula; per element, with t = hp->step >= 1:
+ *   m1 = beta1 m + (1-beta1) g;  v1 = beta2 v + (1-beta2) g^2
+ *   p1 = (1 - lr wd) p - lr (m1 / (1-beta1^t)) / (sqrt(v1 / (1-beta2^t)) + eps)
+ *   P, G: host arrays of n device pointers to tensors of numel[i] elements of
+ *         `dtype` (any shape, contiguous); P is updated in place, G only read.
+ *   M, V: host arrays of n device pointers to numel[i] fp32 moments each,
+ *         updated in place.
+ * No handle and no workspace: the call is stateless (the step count is the
+ * caller's).  16-byte-aligned tensors take the vector path.  Returns
+ * MUON_ERR_INVALID_ARG for null pointers, negative sizes, step < 1, betas
+ * outside [0, 1), eps < 0 or non-finite lr/wd; n == 0 is a no-op.
+ */
+typedef struct {
+  float lr, beta1, beta2, eps, weight_decay;
+  int32_t step;
+} muon_adamw_hparams_t;
+MUON_API muon_status_t muon_adamw_step(void* const* P, const void* const* G, float* const* M, float* const* V,
+                                       const int64_t* numel, int n, muon_dtype_t dtype,
+                                       const muon_adamw_hparams_t* hp, cudaStream_t stream);
+
+/*
  * Copy the n per-matrix Frobenius norms ||U_i||_F of the last step (fp32) into
  * `dst` (host or device memory, n floats), enqueued on `stream`.  Host memory
  * should be pinned for the copy to stay asynchronous.

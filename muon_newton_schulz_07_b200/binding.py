@@ -218,3 +218,20 @@ def muon_momentum_norm_static(G: int, M: int, U: int, rows: int, cols: int, dtyp
     f.restype = ctypes.c_int
     _check(f(ctypes.c_void_p(G), ctypes.c_void_p(M), ctypes.c_void_p(U), int(rows), int(cols), dtype, float(beta),
              1 if nesterov else 0, ctypes.c_void_p(norm), ctypes.c_void_p(stream)), "muon_momentum_norm_static")
+
+
+class AdamWHParams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float), ("step", ctypes.c_int32)]
+
+
+def muon_adamw_step(P, G, M, V, numel, dtype: int, hp: AdamWHParams, stream: int) -> None:
+    L = lib()
+    f = L.muon_adamw_step
+    f.argtypes = [_PP, _PP, _PP, _PP, ctypes.POINTER(ctypes.c_int64), ctypes.c_int, ctypes.c_int,
+                  ctypes.POINTER(AdamWHParams), _VP]
+    f.restype = ctypes.c_int
+    n = len(numel)
+    sizes = (ctypes.c_int64 * max(n, 1))(*[int(x) for x in numel])
+    _check(f(_ptrs(P), _ptrs(G), _ptrs(M), _ptrs(V), sizes, n, dtype, ctypes.byref(hp), ctypes.c_void_p(stream)),
+           "muon_adamw_step")

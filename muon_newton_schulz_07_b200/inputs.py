@@ -127,5 +127,18 @@ def gradient(wl: Workload, step: int, idx: int) -> np.ndarray:
     return normal(wl.wid, step, idx, TID_G, (r, c), 1e-3)
 
 
+# The parameters of the d24 model that AdamW updates.  The magicnetworld page (FLOPs section) gives
+# 1,384,124,976 parameters in all, 679,481,856 in the transformer matrices and 50,331,648 in the
+# lm_head (32768 x 1536); the other 654,311,472 are not itemized there and are modelled as 13
+# embedding tables of 32768 x 1536 plus 48 scalars.
+D24_ADAMW_SIZES = tuple([32768 * 1536] * 14 + [1] * 48)
+
+
+def adamw_param(step: int, idx: int, tid: int, n: int) -> np.ndarray:
+    """Synthetic AdamW tensors: parameters N(0, 0.02^2), gradients N(0, 1e-3^2)."""
+    std = 0.02 if tid == TID_W else 1e-3
+    return normal(100, step, idx, tid, (n,), std)
+
+
 def param_count(wl: Workload) -> int:
     return sum(r * c for r, c in wl.shapes)

@@ -82,3 +82,29 @@ class MuonStep:
             self.close()
         except Exception:
             pass
+
+
+def adamw_step(params, grads, exp_avg, exp_avg_sq, step, lr=1e-3, betas=(0.9, 0.95), eps=1e-8, weight_decay=0.0,
+               stream=None):
+    """AdamW on a list of tensors (bf16 or fp32 parameters, fp32 moments), one fused launch per 256 tensors.
+
+    Every tensor must be contiguous and on the same CUDA device; `step` counts from 1.
+    """
+    if not params:
+        return
+    dt = params[0].dtype
+    if dt not in (torch.bfloat16, torch.float32):
+        raise TypeError("parameters must be bf16 or fp32")
+    for p, g, m, v in zip(params, grads, exp_avg, exp_avg_sq):
+        if not (p.is_contiguous() and g.is_contiguous() and m.is_contiguous() and v.is_contiguous()):
+            raise ValueError("tensors must be contiguous")
+        if p.dtype != dt or g.dtype != dt or m.dtype != torch.float32 or v.dtype != torch.float32:
+            raise ValueError("p, g share the parameter dtype; moments are fp32")
+        if not (p.numel() == g.numel() == m.numel() == v.numel()):
+            raise ValueError("p, g, m, v must have equal sizes")
+    hp = B.AdamWHParams(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay), int(step))
+    s = stream if stream is not None else torch.cuda.current_stream(params[0].device)
+    B.muon_adamw_step([p.data_ptr() for p in params], [g.data_ptr() for g in grads],
+                      [m.data_ptr() for m in exp_avg], [v.data_ptr() for v in exp_avg_sq],
+                      [p.numel() for p in params], B.MUON_BF16 if dt == torch.bfloat16 else B.MUON_FP32, hp,
+                      s.cuda_stream)

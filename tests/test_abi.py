@@ -93,3 +93,17 @@ def test_create_without_device_or_workspace():
     with pytest.raises(B.MuonError) as e:
         B.muon_create([(256, 256)], B.MUON_BF16, B.MUON_MODE_FAST, 1 << 20, 1 << 30)
     assert e.value.code in (B.MUON_ERR_NO_DEVICE, B.MUON_ERR_CUDA)
+
+
+def test_adamw_arguments_checked_on_host():
+    # validation happens before any device work, so this runs without a GPU
+    ok = B.AdamWHParams(1e-3, 0.9, 0.95, 1e-8, 0.0, 1)
+    B.muon_adamw_step([], [], [], [], [], B.MUON_BF16, ok, 0)  # empty: no-op
+    lib = B.lib()
+    bad = B.AdamWHParams(1e-3, 0.9, 0.95, 1e-8, 0.0, 0)  # step counts from 1
+    with pytest.raises(B.MuonError) as e:
+        B.muon_adamw_step([16], [16], [16], [16], [8], B.MUON_BF16, bad, 0)
+    assert e.value.code == B.MUON_ERR_INVALID_ARG
+    with pytest.raises(B.MuonError):
+        B.muon_adamw_step([16], [16], [16], [16], [-1], B.MUON_BF16, ok, 0)
+    assert lib is not None
