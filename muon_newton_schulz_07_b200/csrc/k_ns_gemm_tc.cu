@@ -58,7 +58,6 @@ namespace {
 
 constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK, STAGES = kTcStages;
 constexpr int TILE = 256;                               // pair tile: 256 x 256
-constexpr uint32_t BOX_BYTES = 64 * 64 * 2;             // one TMA box
 constexpr uint32_t A_STAGE = BM * BK * 2;               // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t B_STAGE = (BN / 2) * BK * 2;         // 16 KB: this CTA's half of B
 constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE;     // 32 KB
@@ -155,7 +154,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < p.ngroups; ++g) {
       tma_prefetch_desc(&p.g[g].tm_a);
+      tma_prefetch_desc(&p.g[g].tm_at);
       tma_prefetch_desc(&p.g[g].tm_b);
+      tma_prefetch_desc(&p.g[g].tm_bt);
     }
   }
   if (warp == 1) {
@@ -197,20 +198,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           const bool ta = sym_a && k0 / TILE < ia;
           const bool tb = sym_b && k0 / TILE < jb;
           const bool mnb = ta_update_b || tb;
-          if (!ta) {
+          // One TMA per operand: 128 rows x 64 k (K-major), or 64 k rows x two 64-wide
+          // chunks of the M/N dimension (MN-major), 16 KB each.
+          if (!ta)
             tma_load_3d_pair(sa, &G.tm_a, fb, k0, arow, ti.mat);
-            tma_load_3d_pair(sa + BOX_BYTES, &G.tm_a, fb, k0, arow + 64, ti.mat);
-          } else {
-            tma_load_3d_pair(sa, &G.tm_a, fb, arow, k0, ti.mat);
-            tma_load_3d_pair(sa + BOX_BYTES, &G.tm_a, fb, arow + 64, k0, ti.mat);
-          }
-          if (!mnb) {
+          else
+            tma_load_4d_pair(sa, &G.tm_at, fb, 0, k0, arow / 64, ti.mat);
+          if (!mnb)
             tma_load_3d_pair(sb, &G.tm_b, fb, k0, ti.col0 + half, ti.mat);
-            tma_load_3d_pair(sb + BOX_BYTES, &G.tm_b, fb, k0, ti.col0 + half + 64, ti.mat);
-          } else {
-            tma_load_3d_pair(sb, &G.tm_b, fb, ti.col0 + half, k0, ti.mat);
-            tma_load_3d_pair(sb + BOX_BYTES, &G.tm_b, fb, ti.col0 + half + 64, k0, ti.mat);
-          }
+          else
+            tma_load_4d_pair(sb, &G.tm_bt, fb, 0, k0, (ti.col0 + half) / 64, ti.mat);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;

@@ -40,7 +40,8 @@ struct GroupPlan {
   std::vector<int> mats;      // caller indices, in caller order
   size_t off_x[2], off_a, off_b;
   int scal_base;
-  CUtensorMap tm_x[2], tm_a, tm_b;
+  CUtensorMap tm_x[2], tm_a, tm_b;   // row views (K-major operand tiles)
+  CUtensorMap tt_x[2], tt_a, tt_b;   // chunked views (MN-major operand tiles)
 };
 
 struct Plan {
@@ -158,15 +159,32 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [cnt][rows][cols] bf16, boxes of 64 (cols) x 64 (rows) x 1, 128-byte swizzle.
-bool encode_3d(CUtensorMap* map, void* base, int cols, int rows, int cnt) {
+// Row view of a [cnt][rows][cols] bf16 buffer: one box is 64 columns x 128 rows of one
+// matrix (16 KB, 128-byte swizzle), the K-major operand tile of one CTA and k slice.
+bool encode_rows(CUtensorMap* map, void* base, int cols, int rows, int cnt) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(cnt)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2, static_cast<cuuint64_t>(cols) * rows * 2};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Chunked view of the same buffer, [cnt][cols/64][rows][64]: one box is 64 rows (the k
+// slice) of two neighbouring 64-column chunks, stored chunk after chunk (2 x 8 KB), the
+// MN-major operand tile of one CTA and k slice.
+bool encode_chunks(CUtensorMap* map, void* base, int cols, int rows, int cnt) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(cols / 64),
+                        static_cast<cuuint64_t>(cnt)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(cols) * 2, 128, static_cast<cuuint64_t>(cols) * rows * 2};
+  cuuint32_t box[4] = {64, 64, 2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -367,7 +385,9 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
             const int T = gp.mp / 256;
             if (kind == kGram) {
               G.tm_a = gp.tm_x[cur];
+              G.tm_at = gp.tt_x[cur];
               G.tm_b = gp.tm_x[cur];
+              G.tm_bt = gp.tt_x[cur];
               G.out = h->ws + gp.off_a;
               G.aux = nullptr;
               G.tiles_per_mat = T * (T + 1) / 2;  // 256 x 256 pair tiles on or above the diagonal
@@ -377,7 +397,9 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.m_real = gp.m;
             } else if (kind == kPoly) {
               G.tm_a = gp.tm_a;
+              G.tm_at = gp.tt_a;
               G.tm_b = gp.tm_a;
+              G.tm_bt = gp.tt_a;
               G.out = h->ws + gp.off_b;
               G.aux = h->ws + gp.off_a;
               G.tiles_per_mat = T * (T + 1) / 2;
@@ -387,7 +409,9 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.out_ld = gp.mp;
             } else {
               G.tm_a = gp.tm_b;
+              G.tm_at = gp.tt_b;
               G.tm_b = gp.tm_x[cur];
+              G.tm_bt = gp.tt_x[cur];
               G.out = h->ws + gp.off_x[nxt];
               G.aux = nullptr;
               G.tiles_per_mat = (gp.mp / 256) * (gp.np / 256);  // 256 x 256 pair tiles
@@ -582,10 +606,14 @@ muon_status_t muon_create(muon_handle_t* handle, const muon_shape_t* shapes, int
   }
   if (mode == MUON_MODE_FAST) {
     for (GroupPlan& gp : h->plan.groups) {
-      bool ok = encode_3d(&gp.tm_x[0], h->ws + gp.off_x[0], gp.np, gp.mp, gp.cnt) &&
-                encode_3d(&gp.tm_x[1], h->ws + gp.off_x[1], gp.np, gp.mp, gp.cnt) &&
-                encode_3d(&gp.tm_a, h->ws + gp.off_a, gp.mp, gp.mp, gp.cnt) &&
-                encode_3d(&gp.tm_b, h->ws + gp.off_b, gp.mp, gp.mp, gp.cnt);
+      bool ok = true;
+      for (int b = 0; b < 2; ++b)
+        ok = ok && encode_rows(&gp.tm_x[b], h->ws + gp.off_x[b], gp.np, gp.mp, gp.cnt) &&
+             encode_chunks(&gp.tt_x[b], h->ws + gp.off_x[b], gp.np, gp.mp, gp.cnt);
+      ok = ok && encode_rows(&gp.tm_a, h->ws + gp.off_a, gp.mp, gp.mp, gp.cnt) &&
+           encode_chunks(&gp.tt_a, h->ws + gp.off_a, gp.mp, gp.mp, gp.cnt) &&
+           encode_rows(&gp.tm_b, h->ws + gp.off_b, gp.mp, gp.mp, gp.cnt) &&
+           encode_chunks(&gp.tt_b, h->ws + gp.off_b, gp.mp, gp.mp, gp.cnt);
       if (!ok) {
         delete h;
         return MUON_ERR_CUDA;

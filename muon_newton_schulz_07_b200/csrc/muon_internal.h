@@ -93,8 +93,10 @@ constexpr int kTcThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilog
 enum TcKind : int { kGram = 0, kPoly = 1, kUpdate = 2 };
 
 struct alignas(64) TcGroup {
-  CUtensorMap tm_a;     // operand A source (box 64 x 64 x 1, 128B swizzle)
-  CUtensorMap tm_b;     // operand B source
+  CUtensorMap tm_a;     // operand A source, row view: box 64 (k) x 128 (rows) x 1, 128B swizzle
+  CUtensorMap tm_at;    // the same buffer, chunked view for MN-major reads: box 64 x 64 (k) x 2 chunks x 1
+  CUtensorMap tm_b;     // operand B source, row view
+  CUtensorMap tm_bt;    // operand B source, chunked view
   void* out;            // [cnt][rows][ld] bf16
   const void* aux;      // [cnt][rows][ld] bf16 epilogue input, or nullptr
   int cnt, mp, np;
