@@ -60,21 +60,31 @@ constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK, STAGES = kTcStages;
 constexpr int TILE = 256;                               // pair tile: 256 x 256
 constexpr uint32_t A_STAGE = BM * BK * 2;               // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t B_STAGE = (BN / 2) * BK * 2;         // 16 KB: this CTA's half of B
-constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE;     // 32 KB
 constexpr uint32_t TMEM_COLS = 512;                     // 2 accumulators x 256 fp32 columns
 constexpr uint32_t BAR_BYTES = 256;
-constexpr int EPI_PITCH = 40;                            // staged row: 32 bf16 + 8 pad (80 B, 16-B aligned)
+constexpr int EPI_PITCH = 40;                            // staged aux row: 32 bf16 + 8 pad (80 B, 16-B aligned)
 constexpr int F32_PITCH = 36;                            // staged fp32 row: 32 + 4 pad (144 B, 16-B aligned)
-constexpr uint32_t EPI_WARP_BYTES = 2 * 32 * EPI_PITCH * 2;  // output + auxiliary chunk per warp
-constexpr uint32_t EPI_OFFSET = STAGES * STAGE_BYTES + BAR_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + EPI_OFFSET + 4 * EPI_WARP_BYTES;
-static_assert(32 * F32_PITCH * 4 <= EPI_WARP_BYTES, "fp32 staging must fit the per-warp buffer");
+constexpr int EPI_WARPS = kTcEpiWarps;
+// Shared memory: the stage ring (at most 144 KB: 4 x 32 KB for 256-wide tiles, 3 x 48 KB
+// for 512-wide ones), then per epilogue warp two 32 x 32 bf16 store tiles (2 KB each,
+// 64-byte swizzle), then per warp the auxiliary chunk.  The fp32 staging of the fused
+// parameter write reuses the start of the region (that launch makes no TMA stores).
+constexpr uint32_t STAGE_REGION = 147456;
+constexpr uint32_t EPI_OUT_BYTES = 2048;
+constexpr uint32_t EPI_AUX_BYTES = 32 * EPI_PITCH * 2;
+constexpr uint32_t EPI_F32_BYTES = 32 * F32_PITCH * 4;
+constexpr uint32_t EPI_OFFSET = STAGE_REGION;            // 1024-byte aligned, as the swizzled tiles need
+constexpr uint32_t EPI_AUX_OFFSET = EPI_OFFSET + EPI_WARPS * 2 * EPI_OUT_BYTES;
+constexpr uint32_t BAR_OFFSET = EPI_AUX_OFFSET + EPI_WARPS * EPI_AUX_BYTES;
+constexpr size_t SMEM_BYTES = 1024 + BAR_OFFSET + BAR_BYTES;
+static_assert(EPI_WARPS * EPI_F32_BYTES <= BAR_OFFSET - EPI_OFFSET, "fp32 staging must fit the epilogue region");
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 struct Tile {
   int g, mat, row0, col0;
 };
 
-template <int KIND>
+template <int KIND, int TW>
 __device__ __forceinline__ Tile decode_tile(const TcParams& p, int t) {
   int g = 0;
   while (g + 1 < p.ngroups && p.g[g + 1].tile_begin <= t) ++g;
@@ -88,7 +98,7 @@ __device__ __forceinline__ Tile decode_tile(const TcParams& p, int t) {
   if (KIND == kUpdate) {
     const int tm = r / G.tdim;
     ti.row0 = tm * TILE;
-    ti.col0 = (r - tm * G.tdim) * TILE;
+    ti.col0 = (r - tm * G.tdim) * TW;
   } else {
     // upper-triangle tile q = (I, J), I <= J, row-major over the triangle
     int q = r, I = 0;
@@ -119,19 +129,29 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
   return q;
 }
 
-template <int KIND>
+template <int KIND, bool WIDE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     ns_gemm_tc_kernel(const __grid_constant__ TcParams p) {
+  // WIDE (Update only): the pair tile is 256 x 512, two N = 256 MMAs per k step into one
+  // 512-column accumulator, so every k slice of A feeds twice the columns.
+  constexpr int NSUB = WIDE ? 2 : 1;
+  constexpr int TW = TILE * NSUB;                   // pair tile width
+  constexpr int NST = WIDE ? 3 : STAGES;
+  constexpr uint32_t SB = A_STAGE + NSUB * B_STAGE;  // bytes of one stage in one CTA
+  constexpr int NACC = WIDE ? 1 : 2;                 // accumulators in TMEM
+  static_assert(!WIDE || KIND == kUpdate, "wide tiles are for the Update only");
+  static_assert(NST * SB <= STAGE_REGION, "the stage ring must fit its region");
+  static_assert(NACC * TW <= TMEM_COLS, "accumulators must fit TMEM");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t smem_base = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFFSET);
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
-  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  auto empty_bar = [&](int s) { return bar0 + 8u * (NST + s); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * NST + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * NST + 2 + a); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NST + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -140,13 +160,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   const int ncl = static_cast<int>(num_clusters_x());
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(full_bar(s), 1);   // the even CTA's arrive.expect_tx (bytes of both CTAs)
       mbar_init(empty_bar(s), 1);  // one multicast commit
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf_bar(a), 1);   // one multicast commit
-      mbar_init(acce_bar(a), 8);   // one arrival per epilogue warp of both CTAs
+      mbar_init(acce_bar(a), 2 * EPI_WARPS);   // one arrival per epilogue warp of both CTAs
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -179,7 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       constexpr bool sym_b = KIND == kPoly;
       constexpr bool ta_update_b = KIND == kUpdate;  // X is always read MN-major by Update
       for (int t = cl; t < p.total_tiles; t += ncl) {
-        const Tile ti = decode_tile<KIND>(p, t);
+        const Tile ti = decode_tile<KIND, TW>(p, t);
         const TcGroup& G = p.g[ti.g];
         const int arow = ti.row0 + static_cast<int>(rank) * BM;
         const int ia = ti.row0 / TILE, jb = ti.col0 / TILE;
@@ -189,26 +209,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * SB);
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
-          const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + A_STAGE;
+          const uint32_t sa = smem_base + stage * SB, sb = sa + A_STAGE;
           const int k0 = kb * BK;
           // Blocks of A / B' below the diagonal are not stored: load the transposed block
           // above it instead (the MMA reads it MN-major).
           const bool ta = sym_a && k0 / TILE < ia;
           const bool tb = sym_b && k0 / TILE < jb;
           const bool mnb = ta_update_b || tb;
-          // One TMA per operand: 128 rows x 64 k (K-major), or 64 k rows x two 64-wide
-          // chunks of the M/N dimension (MN-major), 16 KB each.
+          // One TMA per operand tile: 128 rows x 64 k (K-major), or 64 k rows x two 64-wide
+          // chunks of the M/N dimension (MN-major), 16 KB each.  A wide tile has two B
+          // tiles, for tile columns [0, 256) and [256, 512); each CTA holds its half of both.
           if (!ta)
             tma_load_3d_pair(sa, &G.tm_a, fb, k0, arow, ti.mat);
           else
             tma_load_4d_pair(sa, &G.tm_at, fb, 0, k0, arow / 64, ti.mat);
-          if (!mnb)
-            tma_load_3d_pair(sb, &G.tm_b, fb, k0, ti.col0 + half, ti.mat);
-          else
-            tma_load_4d_pair(sb, &G.tm_bt, fb, 0, k0, (ti.col0 + half) / 64, ti.mat);
-          if (++stage == STAGES) {
+#pragma unroll
+          for (int u = 0; u < NSUB; ++u) {
+            const int bcol = ti.col0 + u * TILE + half;
+            if (!mnb)
+              tma_load_3d_pair(sb + u * B_STAGE, &G.tm_b, fb, k0, bcol, ti.mat);
+            else
+              tma_load_4d_pair(sb + u * B_STAGE, &G.tm_bt, fb, 0, k0, bcol / 64, ti.mat);
+          }
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
@@ -217,10 +242,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       }
       // Do not leave while loads or MMAs may still touch this CTA's shared memory:
       // wait (bounded) until the last use of every stage has been released.
-      for (int i = 0; i < STAGES; ++i) {
+      for (int i = 0; i < NST; ++i) {
         if (*abort_flag) break;
         (void)mbar_wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, p.status);
-        if (++stage == STAGES) {
+        if (++stage == NST) {
           stage = 0;
           phase ^= 1u;
         }
@@ -237,11 +262,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = cl; t < p.total_tiles && ok; t += ncl) {
-        const Tile ti = decode_tile<KIND>(p, t);
+        const Tile ti = decode_tile<KIND, TW>(p, t);
         const TcGroup& G = p.g[ti.g];
         if (!mbar_wait_bounded(acce_bar(acc), acc_phase ^ 1u, tmo, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * TW);
         const int ia = ti.row0 / TILE, jb = ti.col0 / TILE;
         for (int kb = 0; kb < G.kblocks; ++kb) {
           if (!mbar_wait_bounded(full_bar(stage), phase, tmo, abort_flag, p.status)) {
@@ -249,7 +274,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + A_STAGE;
+          const uint32_t sa = smem_base + stage * SB, sb = sa + A_STAGE;
           const int kk = kb * BK / TILE;
           const bool mna = sym_a && kk < ia;                        // transposed block of A / B'
           const bool mnb = (KIND == kUpdate) || (sym_b && kk < jb);
@@ -263,37 +288,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           const uint64_t bstep = mnb ? (2048u >> 4) : (32u >> 4);
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j)
-            tc_mma_bf16_pair(d_tmem, adesc0 + astep * j, bdesc0 + bstep * j, idesc, (kb | j) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int u = 0; u < NSUB; ++u)
+              tc_mma_bf16_pair(d_tmem + u * TILE, adesc0 + astep * j, bdesc0 + ((u * B_STAGE) >> 4) + bstep * j, idesc,
+                               (kb | j) != 0 ? 1u : 0u);
           tc_commit_pair_mc(empty_bar(stage), 0x3);  // frees the stage in both CTAs
-          if (++stage == STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
         tc_commit_pair_mc(accf_bar(acc), 0x3);  // accumulator ready for both epilogues
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == NACC) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    // Each warp owns 32 rows of the CTA's 128 (its TMEM lane quadrant) and walks the tile
-    // in 32 x 32 chunks.  A chunk goes through a per-warp shared staging buffer so that
-    // every global access is a run of 64 contiguous bytes: 8 rows x 4 lanes x 16 bytes
-    // per instruction (the auxiliary input, the direct store and the mirrored store).
-    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
-    __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + EPI_OFFSET + (warp - 2) * EPI_WARP_BYTES);
-    __nv_bfloat16* stg_aux = stg + 32 * EPI_PITCH;
+    // Eight warps, two per TMEM lane quadrant: each owns 32 rows of the CTA's 128 and half
+    // of the tile's columns, which it walks in 32 x 32 chunks.  A finished chunk is packed
+    // to bf16 into one of the warp's two 32 x 32 staging tiles (64-byte rows, 64-byte
+    // swizzle, so the row-per-lane writes are free of bank conflicts) and written to global
+    // memory by one TMA store.  The fused parameter write goes through an fp32 staging tile
+    // and plain stores instead, since W is the caller's memory.
+    const int e = warp - 2;                 // epilogue warp 0..7
+    const int quad = warp & 3;              // TMEM lanes 32*quad .. 32*quad+31
+    constexpr int NW = TW / 64;             // chunks per warp and tile
+    const int ch0 = (e >> 2) * NW;          // this warp's first chunk
+    uint8_t* otile = smem + EPI_OFFSET + e * 2 * EPI_OUT_BYTES;
+    const uint32_t otile_u32 = smem_u32(otile);
+    __nv_bfloat16* stg_aux = reinterpret_cast<__nv_bfloat16*>(smem + EPI_AUX_OFFSET + e * EPI_AUX_BYTES);
+    float* st32 = reinterpret_cast<float*>(smem + EPI_OFFSET + e * EPI_F32_BYTES);
     const int sub_r = lane >> 2, sub_c = (lane & 3) * 8;
+    const int swz = (lane >> 1) & 3;  // 64-byte swizzle of this lane's staging row
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = cl; t < p.total_tiles; t += ncl) {
-      const Tile ti = decode_tile<KIND>(p, t);
+      const Tile ti = decode_tile<KIND, TW>(p, t);
       const TcGroup& G = p.g[ti.g];
       const int ld = G.out_ld;
       const size_t mat_off = static_cast<size_t>(ti.mat) * G.mp * ld;
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(G.out) + mat_off;
       const __nv_bfloat16* aux = G.aux ? static_cast<const __nv_bfloat16*>(G.aux) + mat_off : nullptr;
       const int gr0 = ti.row0 + static_cast<int>(rank) * BM + quad * 32;  // first row of this warp
       const int gr = gr0 + lane;
@@ -316,12 +353,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         return tr ? static_cast<size_t>(gc + rr) * ldw + gr0 + sub_c : static_cast<size_t>(gr0 + rr) * ldw + gc + sub_c;
       };
       // The auxiliary input (A for Poly, W for the fused Update) does not depend on the
-      // accumulator: fetch its first chunk (the first at or above the diagonal) before
-      // waiting, and every later chunk one step ahead, so its latency hides behind the
-      // accumulator drain.
+      // accumulator: fetch the warp's first chunk before waiting, and every later chunk
+      // one step ahead, so its latency hides behind the accumulator drain.
       uint4 pf[4];
-      auto pre_load = [&](int c, uint4 (&dst)[4]) {
-        const int gc = ti.col0 + c * 32;
+      auto pre_load = [&](int ch, uint4 (&dst)[4]) {
+        const int gc = ti.col0 + ch * 32;
         if (aux != nullptr) {
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -332,7 +368,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         }
       };
       const bool has_pre = aux != nullptr || wread;
-      if (has_pre) pre_load(0, pf);
+      if (has_pre) pre_load(ch0, pf);
       if (!mbar_wait_bounded(accf_bar(acc), acc_phase, tmo, abort_flag, p.status)) break;
       tc_fence_after();
       float s = 1.0f;
@@ -341,28 +377,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         s = (KIND == kGram) ? al * al : al;
       }
       const float cdiag = (KIND == kPoly && gr < G.m_real) ? p.c_diag : 0.0f;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * TW);
       const uint32_t acce_leader = map_to_rank(acce_bar(acc), 0);
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      for (int c = 0; c < NW; ++c) {
+        const int ch = ch0 + c;
         const int gc0 = ti.col0 + ch * 32;
         float v[32];
         __syncwarp();
         tmem_ld_32cols(taddr + ch * 32, v);
-        if (ch == BN / 32 - 1) {
-          // all of this accumulator has been read: hand it back to the MMA issuer
+        if (c == NW - 1) {
+          // all of this warp's part of the accumulator has been read: tell the MMA issuer
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_remote(acce_leader);
         }
         uint4 nx[4];
-        if (has_pre && ch + 1 < BN / 32) pre_load(ch + 1, nx);
+        if (has_pre && c + 1 < NW) pre_load(ch + 1, nx);
         if (fw) {
           // Last Update: write the parameters instead of X_k.  Chunks in the zero padding
           // of the workspace have no parameters (real dimensions are multiples of 32).
           if (gr0 < G.m_real && gc0 < G.n_real) {
             // stage s * acc in fp32 (row-major, or transposed for tall parameters)
-            float* st32 = reinterpret_cast<float*>(stg);
             if (!tr) {
 #pragma unroll
               for (int i = 0; i < 32; i += 4)
@@ -390,7 +426,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
               }
               __stcs(reinterpret_cast<uint4*>(W + woff(gc0, rr)), pack8(r8));
             }
-            __syncwarp();
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q) pf[q] = nx[q];
@@ -419,20 +454,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (gc0 + i == gr) v[i] += cdiag;
         }
-        // direct store: row-major staging, then 64-byte row runs
-#pragma unroll
-        for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(stg + lane * EPI_PITCH + q * 8) = pack8(v + 8 * q);
+        // The store issued two chunks ago used this staging tile: wait until it has been read.
+        const uint32_t ob = (c & 1) * EPI_OUT_BYTES;
+        if (lane == 0) bulk_wait_read<1>();
         __syncwarp();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int rr = q * 8 + sub_r;
-          *reinterpret_cast<uint4*>(out + static_cast<size_t>(gr0 + rr) * ld + gc0 + sub_c) =
-              *reinterpret_cast<const uint4*>(stg + rr * EPI_PITCH + sub_c);
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(otile + ob + lane * 64 + ((q ^ swz) << 4)) = pack8(v + 8 * q);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&G.tm_out, otile_u32 + ob, gc0, gr0, ti.mat);
+          bulk_commit();
         }
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == NACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
+    // every TMA store of this warp has finished (its shared memory read, its global write)
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   // ------------------------------------------------------------ teardown
@@ -446,16 +489,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   }
 }
 
-template <int KIND>
+template <int KIND, bool WIDE>
 cudaError_t launch_kind(const TcParams& p, int grid, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<KIND, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  ns_gemm_tc_kernel<KIND><<<grid, kTcThreads, SMEM_BYTES, s>>>(p);
+  ns_gemm_tc_kernel<KIND, WIDE><<<grid, kTcThreads, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -467,9 +510,10 @@ cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;
   // one CTA pair per TPC, at most one pair per tile
   const int grid = 2 * std::min(num_sms / 2, p.total_tiles);
-  if (p.kind == kGram) return launch_kind<kGram>(p, grid, s);
-  if (p.kind == kPoly) return launch_kind<kPoly>(p, grid, s);
-  return launch_kind<kUpdate>(p, grid, s);
+  if (p.kind == kGram) return launch_kind<kGram, false>(p, grid, s);
+  if (p.kind == kPoly) return launch_kind<kPoly, false>(p, grid, s);
+  if (p.wide) return launch_kind<kUpdate, true>(p, grid, s);
+  return launch_kind<kUpdate, false>(p, grid, s);
 }
 
 }  // namespace muon

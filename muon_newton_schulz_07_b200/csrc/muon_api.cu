@@ -42,6 +42,7 @@ struct GroupPlan {
   int scal_base;
   CUtensorMap tm_x[2], tm_a, tm_b;   // row views (K-major operand tiles)
   CUtensorMap tt_x[2], tt_a, tt_b;   // chunked views (MN-major operand tiles)
+  CUtensorMap ts_x[2], ts_a, ts_b;   // store views (32 x 32 epilogue tiles)
 };
 
 struct Plan {
@@ -170,6 +171,20 @@ bool encode_rows(CUtensorMap* map, void* base, int cols, int rows, int cnt) {
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Store view of a [cnt][rows][cols] bf16 buffer: one box is a 32 x 32 tile of one matrix
+// (64-byte rows, 64-byte swizzle), one epilogue chunk.
+bool encode_store(CUtensorMap* map, void* base, int cols, int rows, int cnt) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(cnt)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2, static_cast<cuuint64_t>(cols) * rows * 2};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -349,6 +364,14 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
           const int ng = static_cast<int>(std::min<size_t>(kTcMaxGroups, P.groups.size() - g0));
           prm.ngroups = ng;
           prm.kind = kind;
+          // Update takes 256 x 512 pair tiles when every group's padded width allows them:
+          // each k slice of B' then feeds 512 output columns instead of 256.
+          // (The last Update, when it writes the parameters, keeps 256-wide tiles and two
+          // accumulators: its epilogue is too heavy to leave unoverlapped.)
+          bool wide = kind == kUpdate && !(t == k && fuse);
+          for (int gi = 0; gi < ng; ++gi) wide = wide && P.groups[g0 + gi].np % 512 == 0;
+          prm.wide = wide ? 1 : 0;
+          const int tw = wide ? 512 : 256;
           // The first iteration reads the unnormalised U: Gram scales by 1/(||U||+eps)^2 and
           // Update by 1/(||U||+eps); Poly works on the already normalised A.
           prm.use_scal = (t == 1 && kind != kPoly) ? 1 : 0;
@@ -388,6 +411,7 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_at = gp.tt_x[cur];
               G.tm_b = gp.tm_x[cur];
               G.tm_bt = gp.tt_x[cur];
+              G.tm_out = gp.ts_a;
               G.out = h->ws + gp.off_a;
               G.aux = nullptr;
               G.tiles_per_mat = T * (T + 1) / 2;  // 256 x 256 pair tiles on or above the diagonal
@@ -400,6 +424,7 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_at = gp.tt_a;
               G.tm_b = gp.tm_a;
               G.tm_bt = gp.tt_a;
+              G.tm_out = gp.ts_b;
               G.out = h->ws + gp.off_b;
               G.aux = h->ws + gp.off_a;
               G.tiles_per_mat = T * (T + 1) / 2;
@@ -412,11 +437,12 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_at = gp.tt_b;
               G.tm_b = gp.tm_x[cur];
               G.tm_bt = gp.tt_x[cur];
+              G.tm_out = gp.ts_x[nxt];
               G.out = h->ws + gp.off_x[nxt];
               G.aux = nullptr;
-              G.tiles_per_mat = (gp.mp / 256) * (gp.np / 256);  // 256 x 256 pair tiles
+              G.tiles_per_mat = (gp.mp / 256) * (gp.np / tw);  // 256 x tw pair tiles
               G.kblocks = gp.mp / kTcBK;
-              G.tdim = gp.np / 256;
+              G.tdim = gp.np / tw;
               G.out_ld = gp.np;
               G.m_real = gp.m;
               G.n_real = gp.n;
@@ -609,11 +635,14 @@ muon_status_t muon_create(muon_handle_t* handle, const muon_shape_t* shapes, int
       bool ok = true;
       for (int b = 0; b < 2; ++b)
         ok = ok && encode_rows(&gp.tm_x[b], h->ws + gp.off_x[b], gp.np, gp.mp, gp.cnt) &&
-             encode_chunks(&gp.tt_x[b], h->ws + gp.off_x[b], gp.np, gp.mp, gp.cnt);
+             encode_chunks(&gp.tt_x[b], h->ws + gp.off_x[b], gp.np, gp.mp, gp.cnt) &&
+             encode_store(&gp.ts_x[b], h->ws + gp.off_x[b], gp.np, gp.mp, gp.cnt);
       ok = ok && encode_rows(&gp.tm_a, h->ws + gp.off_a, gp.mp, gp.mp, gp.cnt) &&
            encode_chunks(&gp.tt_a, h->ws + gp.off_a, gp.mp, gp.mp, gp.cnt) &&
+           encode_store(&gp.ts_a, h->ws + gp.off_a, gp.mp, gp.mp, gp.cnt) &&
            encode_rows(&gp.tm_b, h->ws + gp.off_b, gp.mp, gp.mp, gp.cnt) &&
-           encode_chunks(&gp.tt_b, h->ws + gp.off_b, gp.mp, gp.mp, gp.cnt);
+           encode_chunks(&gp.tt_b, h->ws + gp.off_b, gp.mp, gp.mp, gp.cnt) &&
+           encode_store(&gp.ts_b, h->ws + gp.off_b, gp.mp, gp.mp, gp.cnt);
       if (!ok) {
         delete h;
         return MUON_ERR_CUDA;

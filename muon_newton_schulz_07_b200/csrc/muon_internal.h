@@ -86,9 +86,10 @@ cudaError_t launch_param_write(const WrParams& p, Dtype io, Dtype xt, cudaStream
 constexpr int kTcBM = 128;
 constexpr int kTcBN = 256;
 constexpr int kTcBK = 64;
-constexpr int kTcStages = 6;
+constexpr int kTcStages = 4;       // 256-wide tiles: 4 x 32 KB; 512-wide tiles: 3 x 48 KB
 constexpr int kTcMaxGroups = 6;
-constexpr int kTcThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kTcEpiWarps = 8;     // two per TMEM lane quadrant, each on half of the tile's columns
+constexpr int kTcThreads = 64 + 32 * kTcEpiWarps;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 
 enum TcKind : int { kGram = 0, kPoly = 1, kUpdate = 2 };
 
@@ -97,6 +98,7 @@ struct alignas(64) TcGroup {
   CUtensorMap tm_at;    // the same buffer, chunked view for MN-major reads: box 64 x 64 (k) x 2 chunks x 1
   CUtensorMap tm_b;     // operand B source, row view
   CUtensorMap tm_bt;    // operand B source, chunked view
+  CUtensorMap tm_out;   // output, store view: box 32 x 32 x 1, 64B swizzle
   void* out;            // [cnt][rows][ld] bf16
   const void* aux;      // [cnt][rows][ld] bf16 epilogue input, or nullptr
   int cnt, mp, np;
@@ -120,6 +122,7 @@ struct TcParams {
   int ngroups;
   int total_tiles;
   int kind;
+  int wide;              // Update with 256 x 512 pair tiles (every group's np a multiple of 512)
   int use_scal;          // first iteration: fold the normalisation in
   float c_acc, c_aux;    // out = s * (c_acc * acc + c_aux * aux) (+ c_diag on the real diagonal)
   float c_diag;

@@ -126,6 +126,32 @@ def test_orthogonalize_shapes(mode, dtype, k):
     print(f"orthogonalize {mode} {dtype} k={k}: " + " ".join(f"{s[0]}x{s[1]}:{e:.2e}" for e, s in errs))
 
 
+# Every group's padded width (max dimension rounded up to 256) is a multiple of 512, so the
+# Update runs on 256 x 512 pair tiles; ragged real sizes leave zero padding inside those tiles.
+WIDE_SHAPES = [(256, 512), (512, 256), (300, 1000), (1000, 300), (512, 1024), (96, 480), (768, 1536)]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("k", [1, 2, 5])
+def test_orthogonalize_wide_update_tiles(dtype, k):
+    rng = np.random.default_rng(17)
+    Xs = [device_tensor(rng.standard_normal(s).astype(np.float32), dtype) for s in WIDE_SHAPES]
+    Os = run_orthogonalize(WIDE_SHAPES, Xs, dtype, "fast", k=k)
+    a, b, c = O.QUINTIC
+    for s, x, o in zip(WIDE_SHAPES, Xs, Os):
+        X = to_f64(x)
+        ref = O.newton_schulz(X, k, O.QUINTIC, 1e-7)
+        if k == 1:
+            smax = np.linalg.norm(X, 2) / np.linalg.norm(X)
+            y = smax * smax
+            amp = abs(b * y + c * y * y) / abs(a + b * y + c * y * y)
+            tol = 2.0 ** -9 * (3.0 + amp) * 1.25
+        else:
+            tol = TOL_O["fast"]
+        tol += out_rounding(dtype)
+        assert rel_fro(to_f64(o), ref) < tol, s
+
+
 def test_intermediates_symmetric_and_padded():
     # Gram and polynomial matrices of the last iteration, read back from the workspace
     # (upper 256 x 256 blocks stored, the rest their transposes): zero outside the real
