@@ -55,6 +55,46 @@ class MuonStep:
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         B.muon_step(self.handle, self._check(W, "W"), self._check(G, "G"), self._check(M, "M"), hp, s.cuda_stream)
 
+    def step_from_host(self, W, G_host, M, stream=None, **hp):
+        """A step whose gradients are in pinned host memory.
+
+        The host-to-device copy of G runs on a side stream into one of two device buffers,
+        so it overlaps the previous step's kernels; the step itself waits for its copy.  The
+        buffer is reused two steps later, once the step that read it has finished.  Keyword
+        arguments are those of __call__.
+        """
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if getattr(self, "_gbuf", None) is None:
+            self._gbuf = [[torch.empty(sh, dtype=self.dtype, device=self.device) for sh in self.shapes]
+                          for _ in range(2)]
+            self._copy_stream = torch.cuda.Stream(self.device)
+            self._buf_free = [None, None]
+            self._nfed = 0
+        if len(G_host) != len(self.shapes):
+            raise ValueError(f"G_host: expected {len(self.shapes)} tensors, got {len(G_host)}")
+        b = self._nfed & 1
+        cs = self._copy_stream
+        with torch.cuda.stream(cs):
+            if self._buf_free[b] is not None:
+                cs.wait_event(self._buf_free[b])
+            for d, h in zip(self._gbuf[b], G_host):
+                if tuple(h.shape) != tuple(d.shape) or h.dtype != d.dtype:
+                    raise ValueError(f"G_host: tensor {tuple(h.shape)} {h.dtype} does not match {tuple(d.shape)} "
+                                     f"{d.dtype}")
+                d.copy_(h, non_blocking=True)
+            copied = torch.cuda.Event()
+            copied.record(cs)
+        s.wait_event(copied)
+        self(W, self._gbuf[b], M, stream=s, **hp)
+        done = torch.cuda.Event()
+        done.record(s)
+        self._buf_free[b] = done
+        self._nfed += 1
+
+    def host_copy_stream(self):
+        """The side stream step_from_host copies on (created by its first call)."""
+        return getattr(self, "_copy_stream", None)
+
     def orthogonalize(self, X, O, eps=1e-7, abc=QUINTIC, ns_steps=5, stream=None):
         hp = B.make_hparams(0.0, 0.0, 0.0, eps, abc, False, ns_steps)
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
