@@ -53,3 +53,30 @@ def test_host_fed_rejects_mismatched_gradients():
     with pytest.raises(ValueError):
         op.step_from_host(W, wrong, M)
     np.testing.assert_array_equal(torch.stack([w.float().abs().sum() for w in W]).cpu().numpy(), 0.0)
+
+
+def test_step_replays_from_a_cuda_graph():
+    # muon_step enqueues kernels and one memset on the caller's stream and never synchronises,
+    # so a captured step replayed twice must equal two eager steps bit for bit.
+    torch.manual_seed(6)
+    dev = torch.device("cuda")
+    W0 = [(torch.randn(s, device=dev) * 0.02).to(torch.bfloat16) for s in SHAPES]
+    M0 = [(torch.randn(s, device=dev) * 1e-3).to(torch.bfloat16) for s in SHAPES]
+    G = [(torch.randn(s, device=dev) * 1e-3).to(torch.bfloat16) for s in SHAPES]
+    We, Me = [w.clone() for w in W0], [m.clone() for m in M0]
+    Wg, Mg = [w.clone() for w in W0], [m.clone() for m in M0]
+    eager, graphed = MuonStep(SHAPES), MuonStep(SHAPES)
+    for _ in range(2):
+        eager(We, G, Me, lr=0.02, beta=0.95)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        graphed(Wg, G, Mg, lr=0.02, beta=0.95, stream=s)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert eager.status() == B.MUON_OK and graphed.status() == B.MUON_OK
+    for we, wg, me, mg in zip(We, Wg, Me, Mg):
+        assert torch.equal(we, wg)
+        assert torch.equal(me, mg)
