@@ -35,7 +35,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["muon", "reference"], default="muon")
-    ap.add_argument("--workload", default="d24", choices=["gpt2s", "d24", "l38b", "stress"])
+    ap.add_argument("--workload", default="d24", choices=["single256", "gpt2s", "d24", "l38b", "stress"])
     ap.add_argument("--ns-steps", type=int, default=5)
     ap.add_argument("--mode", choices=["replica", "sharded"], default="replica",
                     help="replica: every rank steps its own parameter set (weak scaling); sharded: the ranks "
@@ -71,8 +71,9 @@ def flops_by_kind(shapes, k):
 
 def bytes_by_kind(shapes, elem=2):
     n = sum(r * c for r, c in shapes)
-    # momentum_norm: read G, M; write M1 and X0.  write: read W and the final X, write W.
-    return {"momentum_norm": 4 * elem * n, "write": 3 * elem * n}
+    # momentum_norm: read G, M; write M1 (elem bytes each) and the bf16 X0.
+    # write: read W (elem) and the bf16 final X, write W (elem).
+    return {"momentum_norm": (3 * elem + 2) * n, "write": (2 * elem + 2) * n}
 
 
 def measured_traffic(kind, workload):
@@ -282,7 +283,7 @@ def run_muon(args, rank, world, local_rank):
     shapes = list(wl.shapes)
     n = len(shapes)
     k = args.ns_steps
-    dt = torch.bfloat16
+    dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
 
     def to_dev(a):
         return torch.from_numpy(a).to(dev).to(dt)
@@ -397,15 +398,16 @@ def run_muon(args, rank, world, local_rank):
     # ------------------------------------------------------------ roofline
     peaks, peak_src = load_peaks()
     fl = flops_by_kind(shapes, k)
-    by = bytes_by_kind(shapes)
+    by = bytes_by_kind(shapes, 4 if dt == torch.float32 else 2)
     kern = {kname: {"ms_total": ms, "launches": cnt, "ms_per_launch": (ms / cnt if cnt else None)}
             for kname, (ms, cnt) in prof.items() if cnt}
     dominant = max(kern, key=lambda x: kern[x]["ms_total"])
     per_launch_units = {
         "gram": fl["gram"] / k, "poly": fl["poly"] / k, "update": fl["update"] / k,
         "momentum_norm": by["momentum_norm"], "write": by["write"],
+        "ns_small": sum(fl.values()),  # one launch runs every iteration of the step
     }
-    if dominant in ("gram", "poly", "update"):
+    if dominant in ("gram", "poly", "update", "ns_small"):
         ach = per_launch_units[dominant] / (kern[dominant]["ms_per_launch"] * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
@@ -416,11 +418,11 @@ def run_muon(args, rank, world, local_rank):
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "traffic": None, "kernel": dominant, "peak_source": f"{peak_src} hbm_gbs"}
-    ns_ms = sum(kern[x]["ms_total"] for x in ("gram", "poly", "update") if x in kern) / args.steps
+    ns_ms = sum(kern[x]["ms_total"] for x in ("gram", "poly", "update", "ns_small") if x in kern) / args.steps
     ns_flops = sum(fl.values())
     ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms > 0 else None
     for kname, kd in kern.items():
-        if kname in ("gram", "poly", "update"):
+        if kname in ("gram", "poly", "update", "ns_small"):
             kd["tflops"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e12
             kd["frac_of_sustained_peak"] = kd["tflops"] / peaks["bf16_tflops_sustained"]
         elif kname in ("momentum_norm", "write"):

@@ -252,7 +252,8 @@ MUON_API muon_status_t muon_get_group_buffers(muon_handle_t handle, int group, i
 #define MUON_KERNEL_UPDATE 3
 #define MUON_KERNEL_WRITE 4
 #define MUON_KERNEL_SGEMM 5
-#define MUON_KERNEL_KINDS 6
+#define MUON_KERNEL_NS_SMALL 6 /* all iterations of a set of matrices of at most 256 x 256 */
+#define MUON_KERNEL_KINDS 7
 MUON_API muon_status_t muon_profile_begin(muon_handle_t handle, int max_steps);
 MUON_API muon_status_t muon_profile_end(muon_handle_t handle, double* ms, int* launches, int n_kinds);
 

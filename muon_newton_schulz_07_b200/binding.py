@@ -28,7 +28,7 @@ STATUS = {
 MUON_OK, MUON_ERR_INVALID_ARG, MUON_ERR_UNSUPPORTED, MUON_ERR_CUDA = 0, 1, 2, 3
 MUON_ERR_WORKSPACE, MUON_ERR_TIMEOUT, MUON_ERR_DEVICE_STATUS, MUON_ERR_NO_DEVICE = 4, 5, 6, 7
 
-KERNEL_KINDS = ("momentum_norm", "gram", "poly", "update", "write", "sgemm_ref")
+KERNEL_KINDS = ("momentum_norm", "gram", "poly", "update", "write", "sgemm_ref", "ns_small")
 
 
 class MuonError(RuntimeError):

@@ -254,6 +254,7 @@ struct muon_ctx {
   EwParams ew;
   WrParams wr;
   TcParams tc;
+  SmallParams sm;
   // tracing (muon_profile_begin / muon_profile_end)
   int prof_steps_left = 0;
   std::vector<std::pair<int, cudaEvent_t>> prof_events;  // kind (-1: start of a call), event
@@ -338,6 +339,16 @@ cudaError_t enqueue_front(muon_ctx* h, const void* const* src, void* const* mom,
 // The parameter write can ride on the last Update launch when the parameters are bf16,
 // every real dimension is a multiple of 32 (epilogue chunks are all real or all padding),
 // the pointers fit the launch parameters and every destination is 16-byte aligned.
+// All k >= 1 iterations in one kernel when every group pads to one 256 x 256 tile.
+bool small_path(const muon_ctx* h, int k) {
+  if (h->mode != MUON_MODE_FAST || k < 1 || h->plan.groups.empty() ||
+      h->plan.groups.size() > static_cast<size_t>(kTcMaxGroups))
+    return false;
+  for (const GroupPlan& gp : h->plan.groups)
+    if (gp.mp != kSmallTile || gp.np != kSmallTile) return false;
+  return true;
+}
+
 bool write_fusable(const muon_ctx* h, void* const* dst, int k) {
   if (h->mode != MUON_MODE_FAST || h->dtype != MUON_BF16 || k < 1 || !h->fuse_shapes_ok) return false;
   for (int i = 0; i < h->n; ++i)
@@ -352,6 +363,39 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
                        bool store_only, bool* fused) {
   const Plan& P = h->plan;
   const int k = hp->ns_steps;
+  if (small_path(h, k)) {
+    // every matrix fits one 256 x 256 tile: all k iterations in one launch, X_k into X[k & 1]
+    *fused = false;
+    SmallParams& sp = h->sm;
+    std::memset(&sp, 0, sizeof(sp));
+    int mats = 0;
+    for (size_t g = 0; g < P.groups.size(); ++g) {
+      const GroupPlan& gp = P.groups[g];
+      SmGroup& G = sp.g[g];
+      G.tm_row = gp.tm_x[0];
+      G.tm_col = gp.tt_x[0];
+      G.out = h->ws + gp.off_x[k & 1];
+      G.mat_begin = mats;
+      G.cnt = gp.cnt;
+      G.scal_base = gp.scal_base;
+      G.m_real = gp.m;
+      mats += gp.cnt;
+    }
+    sp.ngroups = static_cast<int>(P.groups.size());
+    sp.total = mats;
+    sp.k = k;
+    sp.a = hp->a;
+    sp.b = hp->b;
+    sp.c = hp->c;
+    sp.scal = h->d_scal;
+    sp.status = h->d_status;
+    sp.timeout_ns = kTimeoutNs;
+    cudaError_t e = launch_ns_small(sp, h->num_sms, st);
+    if (e != cudaSuccess) return e;
+    ++*launches;
+    trace(h, MUON_KERNEL_NS_SMALL, st);
+    return cudaSuccess;
+  }
   const bool fuse = write_fusable(h, dst, k);
   *fused = fuse;
   for (int t = 1; t <= k; ++t) {
@@ -551,6 +595,7 @@ cudaError_t enqueue_back(muon_ctx* h, void* const* dst, const muon_hparams_t* hp
 
 int launches_for(const muon_ctx* h, int k) {
   const int chunks = (h->n + kEwMatsPerLaunch - 1) / kEwMatsPerLaunch;
+  if (small_path(h, k)) return chunks + 1 + chunks;
   const int ng = static_cast<int>(h->plan.groups.size());
   const int per_stage = (h->mode == MUON_MODE_FAST) ? (ng + kTcMaxGroups - 1) / kTcMaxGroups : ng;
   const bool fused = h->mode == MUON_MODE_FAST && h->dtype == MUON_BF16 && k >= 1 && h->fuse_shapes_ok;

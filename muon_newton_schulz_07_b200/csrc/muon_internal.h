@@ -143,6 +143,35 @@ struct TcParams {
 size_t tc_smem_bytes();
 cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s);
 
+// ------------------------------------------------------------------ small matrices, all iterations in one kernel
+// Every matrix of the set fits one 256 x 256 tile (max(rows, cols) <= 256; the workspace
+// pads it to 256 x 256).  One CTA pair runs all k Newton-Schulz iterations of a matrix.
+constexpr int kSmallTile = 256;
+
+struct alignas(64) SmGroup {
+  CUtensorMap tm_row;   // X0, row view (box 64 x 128 x 1): this CTA's 128 rows, one 64-wide k chunk
+  CUtensorMap tm_col;   // X0, chunked view (box 64 x 64 x 2 x 1): 64 rows of this CTA's 128 columns
+  void* out;            // [cnt][256][256] bf16: X_k
+  int mat_begin;        // first matrix of the group in the launch's numbering
+  int cnt;
+  int scal_base;
+  int m_real;           // real rows of the Gram matrix (the polynomial's a I stops there)
+};
+
+struct SmallParams {
+  SmGroup g[kTcMaxGroups];
+  int ngroups;
+  int total;            // matrices in the launch
+  int k;                // Newton-Schulz iterations, >= 1
+  float a, b, c;
+  const float* scal;    // per matrix {||U||, 1/(||U||+eps)}
+  unsigned int* status;
+  unsigned long long timeout_ns;
+};
+
+size_t small_smem_bytes();
+cudaError_t launch_ns_small(const SmallParams& p, int num_sms, cudaStream_t s);
+
 // ------------------------------------------------------------------ fp32 reference GEMMs
 struct SgParams {
   const float* a; const float* b; float* c; const float* aux;
