@@ -49,6 +49,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "muon_device.cuh"
 #include "muon_internal.h"
@@ -491,12 +492,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
 
 template <int KIND, bool WIDE>
 cudaError_t launch_kind(const TcParams& p, int grid, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<KIND, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(SMEM_BYTES));
+  // The shared-memory limit is a property of the function on each device: set it once per device.
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if ((attr_set.load() & bit) == 0) {
+    e = cudaFuncSetAttribute(ns_gemm_tc_kernel<KIND, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set.fetch_or(bit);
   }
   ns_gemm_tc_kernel<KIND, WIDE><<<grid, kTcThreads, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();

@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "muon_device.cuh"
 #include "muon_internal.h"
@@ -250,12 +251,17 @@ size_t small_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_ns_small(const SmallParams& p, int num_sms, cudaStream_t s) {
   if (p.total <= 0) return cudaSuccess;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(SMEM_BYTES));
+  // The shared-memory limit is a property of the function on each device: set it once per device.
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if ((attr_set.load() & bit) == 0) {
+    e = cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set.fetch_or(bit);
   }
   const int grid = 2 * std::min(num_sms / 2, p.total);
   ns_small_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(p);
