@@ -228,8 +228,10 @@ def run_reference(args, rank):
     times = {s: [] for s in shapes}
     t_begin = time.perf_counter()
     done = 0
-    for it in range(args.warmup + args.steps):
-        s = shapes[it % len(shapes)]
+    # the timed steps start over at the first shape and cover every shape at least once
+    n_timed = max(args.steps, len(shapes))
+    for it in range(args.warmup + n_timed):
+        s = shapes[(it if it < args.warmup else it - args.warmup) % len(shapes)]
         i = first[s]
         W, G, M = (I.weight(wl, i).astype(np.float64), I.gradient(wl, 1 + it, i).astype(np.float64),
                    I.momentum(wl, i).astype(np.float64))
