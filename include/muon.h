@@ -28,6 +28,16 @@
  * work has finished.  Calls on one handle must not overlap on the device
  * (they share the workspace).
  *
+ * Kernels.  A step enqueues the momentum/norm kernel, then the Newton-Schulz
+ * iterations, then the parameter write.  In MUON_MODE_FAST the iterations run
+ * as three tensor-core launches each (Gram, polynomial, update) over every
+ * matrix of the handle, with the parameter write fused into the last update
+ * for bf16 sets whose dimensions are multiples of 32.  When every matrix fits
+ * one 256 x 256 tile (max(rows, cols) <= 256, at most six distinct shapes),
+ * all k iterations run in one launch instead (MUON_KERNEL_NS_SMALL).
+ * Results are the same function of the inputs on either path, within the
+ * bf16 rounding described under muon_mode_t.
+ *
  * Errors.  Every entry point returns a muon_status_t and never throws.
  * Argument errors are detected on the host before anything is enqueued.
  * Launch failures return MUON_ERR_CUDA.  Faults the kernels detect on the
@@ -67,9 +77,11 @@ typedef enum { MUON_BF16 = 0, MUON_FP32 = 1 } muon_dtype_t;
 
 /* Arithmetic of the Newton-Schulz products.
  * FAST:     bf16 operands on the tcgen05 tensor cores, fp32 accumulation in
- *           TMEM, fp32 epilogue math, bf16 intermediates X, A, B.
- * FP32_REF: fp32 operands and fp32 FMA on the CUDA cores (no TF32), fp32
- *           intermediates: a slow, accurate mode for checking. */
+ *           TMEM, fp32 epilogue math, one bf16 rounding per stored intermediate
+ *           (X, A, and B' = a I + b A + c A A, every term of B' taken from the
+ *           rounded A).
+ * FP32_REF: fp32 operands and intermediates, products accumulated in fp64 on
+ *           the CUDA cores (no TF32): a slow, accurate mode for checking. */
 typedef enum { MUON_MODE_FAST = 0, MUON_MODE_FP32_REF = 1 } muon_mode_t;
 
 typedef struct { int64_t rows, cols; } muon_shape_t;
