@@ -1,0 +1,77 @@
+"""The measurement code of bench.py that runs on the host: work counts, the traffic record and
+the reference arm's sampling.  CPU only."""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import shutil
+
+import numpy as np
+import pytest
+
+import bench
+import oracle as O
+from muon_newton_schulz_07_b200 import inputs as I
+
+
+@pytest.mark.parametrize("name", ["single256", "gpt2s", "d24", "l38b"])
+def test_flop_counts_match_the_oracle_definition(name):
+    wl = I.WORKLOADS[name]
+    fl = bench.flops_by_kind(wl.shapes, 5)
+    assert sum(fl.values()) == sum(O.ns_flops(r, c, 5) for r, c in wl.shapes)
+    m, n = 1536, 6144
+    one = bench.flops_by_kind([(m, n)], 1)
+    assert one == {"gram": m * m * n, "poly": m ** 3, "update": 2 * m * m * n}
+
+
+def test_byte_counts_per_element():
+    shapes = [(3, 5), (7, 2)]
+    n = 3 * 5 + 7 * 2
+    # bf16 storage: G, M in, M1 out, bf16 X0 out; W in, bf16 X_k in, W out
+    assert bench.bytes_by_kind(shapes, 2) == {"momentum_norm": 8 * n, "write": 6 * n}
+    # fp32 storage: the same tensors at 4 bytes, X stays bf16
+    assert bench.bytes_by_kind(shapes, 4) == {"momentum_norm": 14 * n, "write": 10 * n}
+
+
+def test_traffic_record_is_used_only_for_the_captured_source(tmp_path, monkeypatch):
+    rec_path = os.path.join(bench.ROOT, "profiles", "traffic_update_d24.json")
+    with open(rec_path) as f:
+        rec = json.load(f)
+    got = bench.measured_traffic("update", "d24")
+    assert got == (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * rec["scale_to_workload"]["d24"]
+    assert bench.measured_traffic("update", "gpt2s") is None  # no capture for that workload
+    assert bench.measured_traffic("gram", "d24") is None      # no record for that kernel
+    # a changed kernel source invalidates the record
+    root = tmp_path / "repo"
+    shutil.copytree(os.path.join(bench.ROOT, "profiles"), root / "profiles")
+    src = root / rec["source"]
+    src.parent.mkdir(parents=True)
+    src.write_text("// a different kernel\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.measured_traffic("update", "d24") is None
+
+
+def test_reference_arm_times_every_shape_even_on_short_runs(monkeypatch, capsys):
+    calls = []
+
+    def fake_step(W, G, M, hp):
+        calls.append(W.shape)
+        return W, M, W
+
+    monkeypatch.setattr(O, "muon_step", fake_step)
+    args = argparse.Namespace(workload="d24", steps=1, warmup=1, ns_steps=5, gpus=1, reference_budget_s=150.0)
+    bench.run_reference(args, rank=0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    shapes = sorted(set(I.WORKLOADS["d24"].shapes))
+    assert sorted(set(calls)) == shapes           # every distinct shape was stepped
+    assert line["steps"] >= len(shapes) and line["impl"] == "reference"
+    assert line["value"] > 0 and np.isfinite(line["value"])
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_is_silent_on_other_ranks(capsys):
+    args = argparse.Namespace(workload="d24", steps=1, warmup=1, ns_steps=5, gpus=2, reference_budget_s=1.0)
+    bench.run_reference(args, rank=1)
+    assert capsys.readouterr().out == ""
