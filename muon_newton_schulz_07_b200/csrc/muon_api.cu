@@ -9,7 +9,9 @@
 //   k x { Gram, Poly, Update }   tcgen05 kernels, every shape group in one launch
 //                                (or fp32 CUDA-core kernels, one per group, in
 //                                the reference mode); the last Update writes the
-//                                parameters itself when the shapes allow it
+//                                parameters itself when the shapes allow it.  When
+//                                every matrix fits one 256 x 256 tile, one
+//                                ns_small_kernel launch runs all k iterations instead.
 //   param_write_kernel     (one launch per <= 192 matrices, only when not fused)
 #include <algorithm>
 #include <cmath>
