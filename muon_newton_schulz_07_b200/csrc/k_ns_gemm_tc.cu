@@ -27,19 +27,29 @@
 // stored block above it and feeds it to the tensor core as an MN-major operand,
 // so the lower halves of A and B' are never written or read.
 //
-// Roles in each CTA (192 threads, one CTA per SM, persistent over a static
+// Wide Update tiles.  When every group's padded width is a multiple of 512, the
+// Updates that do not write the parameters use 256 x 512 pair tiles: two N = 256
+// MMAs per k step share each k slice of B', so 25 % fewer operand bytes cross from
+// L2 per multiply-add, at the price of one 512-column accumulator (the epilogue
+// of a tile no longer overlaps the main loop of the next).
+//
+// Roles in each CTA (320 threads, one CTA per SM, persistent over a static
 // round-robin list of pair tiles):
-//   warp 0      TMA producer into a 6-stage ring of {A 128 x 64, B 128 x 64}
-//               bf16 tiles (64 x 64 boxes, 128-byte swizzle); the even CTA's
-//               full barrier counts the bytes of both CTAs
+//   warp 0      TMA producer, one TMA per operand tile and k slice (a 64 x 128
+//               box for K-major tiles, a 4-D box of two 64-wide chunks for
+//               MN-major ones, 128-byte swizzle) into a ring of 4 stages of
+//               32 KB (3 of 48 KB for wide tiles); the even CTA's full barrier
+//               counts the bytes of both CTAs
 //   warp 1      TMEM allocation (512 columns: two 256-column accumulators, so
-//               the epilogue of one tile overlaps the main loop of the next);
-//               in the even CTA, lane 0 issues the MMAs
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, the fp32 combination
-//               (Poly: c A A + b A + a I), bf16 cast, stores staged through
-//               shared memory so every global access is a 64-byte row run
-//               (upper blocks only for Gram/Poly).  In the last Update
-//               the epilogue writes the parameters directly:
+//               the epilogue of one tile overlaps the main loop of the next, or
+//               one 512-column accumulator for wide tiles); in the even CTA,
+//               lane 0 issues the MMAs
+//   warps 2..9  epilogue, two warps per TMEM lane quadrant, each on half of the
+//               tile's columns: tcgen05.ld 32 columns at a time, the fp32
+//               combination (Poly: c A A + b A + a I), bf16 pack into a
+//               64B-swizzled 32 x 32 staging tile, one TMA store per chunk
+//               (upper blocks only for Gram/Poly).  In the last Update the
+//               epilogue writes the parameters directly:
 //               W = (1 - lr wd) W - lr sqrt(max(1, r/c)) X_k from the unrounded
 //               fp32 X_k, transposed back for tall matrices.
 // Operand B of Update is X itself in its row-major layout, i.e. MN-major, and so
