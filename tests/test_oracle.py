@@ -329,3 +329,60 @@ def test_adamw_pin_catches_missing_bias_correction():
     right = O.adamw_step(np.zeros(10), g, np.zeros(10), np.zeros(10), 1, lr=1e-2, beta1=0.9, beta2=0.95,
                          eps=1e-8, weight_decay=0.0)[0]
     assert np.max(np.abs(right - wrong)) > 1e-3
+
+
+def _step_orientation_pin_holds():
+    # Stepping the transposed matrix gives the transposed M1 and direction O exactly; only the
+    # shape scale changes, since it is taken on the caller's own orientation:
+    # (W1 - (1 - lr wd) W) / (-lr sqrt(max(1, r/c))) = O for either orientation.
+    rng = np.random.default_rng(31)
+    r, c = 24, 10  # tall: the oracle orthogonalises its transpose and transposes back
+    W, G, M = (rng.standard_normal((r, c)) for _ in range(3))
+    hp = O.Hyper(lr=0.05, beta=0.9, weight_decay=0.2, eps=1e-7, nesterov=True, ns_steps=4)
+    W1, M1, O1 = O.muon_step(W, G, M, hp)
+    W1t, M1t, O1t = O.muon_step(W.T, G.T, M.T, hp)
+    decay = 1.0 - hp.lr * hp.weight_decay
+    d = (W1 - decay * W) / (-hp.lr * np.sqrt(r / c))
+    dt = (W1t - decay * W.T) / (-hp.lr * 1.0)
+    return (np.array_equal(M1t, M1.T) and np.array_equal(O1t, O1.T) and rel(d, O1) < 1e-13
+            and rel(dt, O1t) < 1e-13)
+
+
+def test_full_step_transpose_equivariance():
+    assert _step_orientation_pin_holds()
+    rng = np.random.default_rng(31)
+    r, c = 24, 10
+    W, G, M = (rng.standard_normal((r, c)) for _ in range(3))
+    # the direction of a tall matrix has orthonormal-ish columns: O^T O near I after enough steps
+    hp_many = O.Hyper(lr=0.05, beta=0.9, weight_decay=0.0, eps=1e-7, nesterov=True, ns_steps=60, abc=O.CUBIC)
+    _, _, Oc = O.muon_step(W, G, M, hp_many)
+    assert rel(Oc.T @ Oc, np.eye(c)) < 1e-6
+
+
+def test_full_step_without_nesterov_orthogonalises_the_momentum():
+    rng = np.random.default_rng(32)
+    W, G, M = (rng.standard_normal((6, 9)) for _ in range(3))
+    hp = O.Hyper(lr=0.1, beta=0.8, weight_decay=0.0, eps=1e-7, nesterov=False, ns_steps=3)
+    _, M1, O1 = O.muon_step(W, G, M, hp)
+    # without the Nesterov blend the direction is NS(M1), not NS((1 - beta) G + beta M1)
+    assert rel(O1, O.newton_schulz(M1, 3)) < 1e-14
+    hp_n = O.Hyper(lr=0.1, beta=0.8, weight_decay=0.0, eps=1e-7, nesterov=True, ns_steps=3)
+    _, _, On = O.muon_step(W, G, M, hp_n)
+    assert rel(On, O1) > 1e-3
+
+
+def test_step_pin_catches_planted_mistakes(monkeypatch):
+    import math
+
+    import oracle.muon_oracle as mo
+
+    assert _step_orientation_pin_holds()
+    # the shape scale taken on the oriented (min x max) shape instead of the caller's
+    with monkeypatch.context() as mp:
+        mp.setattr(mo, "shape_scale", lambda r, c: math.sqrt(max(r, c) / min(r, c)))
+        assert not _step_orientation_pin_holds()
+    # weight decay applied after the update instead of to the pre-update W
+    with monkeypatch.context() as mp:
+        mp.setattr(mo, "parameter_write",
+                   lambda W, Ov, lr, wd: (1.0 - lr * wd) * (W - lr * mo.shape_scale(*W.shape) * Ov))
+        assert not _step_orientation_pin_holds()
