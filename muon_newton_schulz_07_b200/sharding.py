@@ -77,9 +77,48 @@ class ShardedMuon:
         self.local_step = local_step
 
     def step(self, W, G, M_owned, **hp):
+        """A step from gradients already averaged over the ranks (G: the full list on every rank)."""
         if self.owned:
             self.local_step([W[i] for i in self.owned], [G[i] for i in self.owned], M_owned, **hp)
         self.exchange(W)
+
+    def step_local_grads(self, W, G_local, M_owned, **hp):
+        """A data-parallel step from this rank's own gradients: average them over the ranks by a
+        reduce-scatter that hands each rank only the matrices it owns, step those, all-gather W."""
+        G_owned = self.reduce_gradients(G_local)
+        if self.owned:
+            self.local_step([W[i] for i in self.owned], G_owned, M_owned, **hp)
+        self.exchange(W)
+
+    def reduce_gradients(self, G_local):
+        """The mean over the ranks of the owned matrices' gradients, in owned order.
+
+        Every rank packs its full list of local gradients into one buffer, rank q's owned matrices
+        in segment q (segments padded to the longest); one reduce-scatter sums segment q onto rank
+        q, which divides by the number of ranks.  The sum runs in the gradients' dtype.  This is
+        the collective that replaces a replicated trainer's all-reduce: each rank receives 1/N of
+        the data instead of all of it.  The returned tensors are views of one fresh buffer.
+        """
+        if self.world == 1:
+            return [G_local[i] for i in self.owned]
+        ref = G_local[0]
+        longest = max(self.sizes)
+        send = torch.zeros(self.world * longest, dtype=ref.dtype, device=ref.device)
+        for q in range(self.world):
+            off = q * longest
+            for i in self.by_rank[q]:
+                n = G_local[i].numel()
+                send[off:off + n].copy_(G_local[i].reshape(-1))
+                off += n
+        recv = torch.empty(longest, dtype=ref.dtype, device=ref.device)
+        dist.reduce_scatter_tensor(recv, send, op=dist.ReduceOp.SUM, group=self.group)
+        recv.div_(self.world)
+        out, off = [], 0
+        for i in self.owned:
+            n = G_local[i].numel()
+            out.append(recv[off:off + n].view_as(G_local[i]))
+            off += n
+        return out
 
     def exchange(self, W):
         """Every rank gets the parameters its peers own: one all-gather of packed, padded shards."""

@@ -92,3 +92,46 @@ def test_sharded_step_equals_unsharded_world2():
                 assert np.array_equal(z[f"m{i}"], ref[i][1])
             owned_all += list(z["owned"])
         assert sorted(owned_all) == list(range(len(SHAPES)))
+
+
+def _local_grad(rank, G):
+    # each rank's own gradient: the shared part plus a rank-dependent part
+    rng = np.random.default_rng(100 + rank)
+    return [g + torch.from_numpy(rng.standard_normal(tuple(g.shape))) for g in G]
+
+
+def _worker_local_grads(rank, world, port, outdir):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        W, G, M = _inputs()
+        sh = ShardedMuon(SHAPES, rank, world, local_step=_oracle_local_step)
+        M_owned = [M[i] for i in sh.owned]
+        sh.step_local_grads(W, _local_grad(rank, G), M_owned, **HP)
+        np.savez(os.path.join(outdir, f"rank{rank}.npz"), *[w.numpy() for w in W], owned=np.array(sh.owned),
+                 **{f"m{i}": M[i].numpy() for i in sh.owned})
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_scatter_step_equals_unsharded_step_on_the_mean_gradient():
+    # Each rank brings its own gradients; the sharded step averages them by a reduce-scatter over
+    # the ownership, steps its own matrices and all-gathers W.  The result must be the unsharded
+    # step on the mean gradient, bit for bit (two float64 summands: the sum and the halving are exact).
+    world = 2
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_worker_local_grads, args=(world, _free_port(), d), nprocs=world, join=True,
+                           start_method="spawn")
+        W, G, M = _inputs()
+        locals_ = [_local_grad(r, G) for r in range(world)]
+        G_mean = [(a + b) / 2 for a, b in zip(*locals_)]
+        hp = O.Hyper(**{k: v for k, v in HP.items()})
+        ref = [O.muon_step(w.numpy(), g.numpy(), m.numpy(), hp) for w, g, m in zip(W, G_mean, M)]
+        owned_all = []
+        for r in range(world):
+            z = np.load(os.path.join(d, f"rank{r}.npz"))
+            for i in range(len(SHAPES)):
+                assert np.array_equal(z[f"arr_{i}"], ref[i][0]), (r, i)
+            for i in z["owned"]:
+                assert np.array_equal(z[f"m{i}"], ref[i][1])
+            owned_all += list(z["owned"])
+        assert sorted(owned_all) == list(range(len(SHAPES)))
