@@ -24,6 +24,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "muon.h"
 #include "muon_internal.h"
@@ -33,6 +34,15 @@ using namespace muon;
 namespace {
 
 constexpr unsigned long long kTimeoutNs = 4000000000ull;  // bounded waits give up after 4 s
+
+// An NVTX range around the host-side enqueue of a call or a stage: it names the stages on a
+// profiler's timeline and costs nothing when no profiler is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int round_up(long long x, int a) { return static_cast<int>((x + a - 1) / a * a); }
@@ -285,6 +295,7 @@ void trace_call_end(muon_ctx* h) {
 // The elementwise front end (momentum + norm + orientation) over all matrices.
 cudaError_t enqueue_front(muon_ctx* h, const void* const* src, void* const* mom, const muon_hparams_t* hp,
                           cudaStream_t st, int* launches) {
+  NvtxRange range("muon: momentum + norm");
   const Plan& P = h->plan;
   const Dtype io = (h->dtype == MUON_BF16) ? kBF16 : kF32;
   const Dtype xt = (h->mode == MUON_MODE_FAST) ? kBF16 : kF32;
@@ -367,6 +378,7 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
   const int k = hp->ns_steps;
   if (small_path(h, k)) {
     // every matrix fits one 256 x 256 tile: all k iterations in one launch, X_k into X[k & 1]
+    NvtxRange range("muon: Newton-Schulz, all iterations (small matrices)");
     *fused = false;
     SmallParams& sp = h->sm;
     std::memset(&sp, 0, sizeof(sp));
@@ -404,6 +416,7 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
     const int cur = (t - 1) & 1, nxt = t & 1;
     if (h->mode == MUON_MODE_FAST) {
       for (int kind = kGram; kind <= kUpdate; ++kind) {
+        NvtxRange range(kind == kGram ? "muon: Gram" : kind == kPoly ? "muon: polynomial" : "muon: update");
         for (size_t g0 = 0; g0 < P.groups.size(); g0 += kTcMaxGroups) {
           TcParams& prm = h->tc;
           std::memset(&prm, 0, sizeof(prm));
@@ -504,6 +517,7 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
       }
     } else {
       for (int kind = kGram; kind <= kUpdate; ++kind) {
+        NvtxRange range(kind == kGram ? "muon: Gram" : kind == kPoly ? "muon: polynomial" : "muon: update");
         for (const GroupPlan& gp : P.groups) {
           SgParams s{};
           const float* x = reinterpret_cast<const float*>(h->ws + gp.off_x[cur]);
@@ -550,6 +564,7 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
 
 cudaError_t enqueue_back(muon_ctx* h, void* const* dst, const muon_hparams_t* hp, bool store_only, cudaStream_t st,
                          int* launches) {
+  NvtxRange range("muon: parameter write");
   const Plan& P = h->plan;
   const Dtype io = (h->dtype == MUON_BF16) ? kBF16 : kF32;
   const Dtype xt = (h->mode == MUON_MODE_FAST) ? kBF16 : kF32;
@@ -712,6 +727,7 @@ muon_status_t muon_step(muon_handle_t h, void* const* W, const void* const* G, v
   for (int i = 0; i < h->n; ++i)
     if (W[i] == nullptr || G[i] == nullptr || M[i] == nullptr) return MUON_ERR_INVALID_ARG;
   DeviceGuard guard(h->device);
+  NvtxRange range("muon_step");
   int launches = 0;
   bool fused = false;
   cudaError_t e = enqueue_front(h, G, M, hp, stream, &launches);
@@ -727,6 +743,7 @@ muon_status_t muon_orthogonalize(muon_handle_t h, const void* const* X, void* co
   for (int i = 0; i < h->n; ++i)
     if (X[i] == nullptr || O[i] == nullptr) return MUON_ERR_INVALID_ARG;
   DeviceGuard guard(h->device);
+  NvtxRange range("muon_orthogonalize");
   muon_hparams_t q = *hp;
   q.beta = 0.0f;
   q.nesterov = 0;
