@@ -386,3 +386,27 @@ def test_step_pin_catches_planted_mistakes(monkeypatch):
         mp.setattr(mo, "parameter_write",
                    lambda W, Ov, lr, wd: (1.0 - lr * wd) * (W - lr * mo.shape_scale(*W.shape) * Ov))
         assert not _step_orientation_pin_holds()
+
+
+def test_adamw_weight_decay_is_decoupled(monkeypatch):
+    # g = 0 with fresh moments: m1 = v1 = 0, so the Adam update is exactly 0 and only the decoupled
+    # decay acts, p1 = (1 - lr wd) p.  Adding wd p to the gradient instead (Adam with L2) would
+    # move the moments and fail this.
+    import oracle.muon_oracle as mo
+
+    p = np.array([1.5, -2.0, 0.25, 3.0])
+    z = np.zeros_like(p)
+    p1, m1, v1 = O.adamw_step(p, z, z, z, 1, lr=0.01, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1)
+    assert np.array_equal(m1, z) and np.array_equal(v1, z)
+    assert np.max(np.abs(p1 - (1.0 - 0.01 * 0.1) * p)) < 1e-16
+
+    def l2_in_gradient(p, g, m, v, step, lr, beta1, beta2, eps, weight_decay):
+        g = g + weight_decay * p
+        m1 = beta1 * m + (1 - beta1) * g
+        v1 = beta2 * v + (1 - beta2) * g * g
+        mh, vh = m1 / (1 - beta1 ** step), v1 / (1 - beta2 ** step)
+        return p - lr * mh / (np.sqrt(vh) + eps), m1, v1
+
+    monkeypatch.setattr(mo, "adamw_step", l2_in_gradient)
+    q1, _, _ = mo.adamw_step(p, z, z, z, 1, lr=0.01, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1)
+    assert np.max(np.abs(q1 - (1.0 - 0.01 * 0.1) * p)) > 1e-3
