@@ -247,6 +247,34 @@ def test_gpt2s_orthogonal_direction():
 
 # ---------------------------------------------------------------- determinism, resume, failure detection
 
+def test_gpt2s_free_running_drift():
+    # Ten steps with no teacher forcing: the GPU state and the oracle's (float64 from the same bf16
+    # start, the same bf16 gradients) drift apart only through the per-step roundings.  W is stored
+    # in bf16 every step (2^-9 relative) and M carries a 0.95 memory of its own roundings, so ten
+    # steps stay near 1e-2; the drift is printed and held to 5e-2 (a wrong formula gives O(1)).
+    wl = I.WORKLOADS["gpt2s"]
+    idx = [0, 4, 5, 6, 10, 11]
+    shapes = [wl.shapes[i] for i in idx]
+    W, G, M = workload_tensors(wl, torch.bfloat16, step=1, idx=idx)
+    Wr, Mr = [to_f64(w) for w in W], [to_f64(m) for m in M]
+    op = MuonStep(shapes, dtype=torch.bfloat16)
+    hp = oracle_hp()
+    steps = 10
+    for step in range(1, steps + 1):
+        if step > 1:
+            G = [device_tensor(I.gradient(wl, step, i), torch.bfloat16) for i in idx]
+        Gr = [to_f64(g) for g in G]
+        op(W, G, M, lr=0.02, beta=0.95, ns_steps=5)
+        for j in range(len(idx)):
+            Wr[j], Mr[j], _ = O.muon_step(Wr[j], Gr[j], Mr[j], hp)
+    torch.cuda.synchronize()
+    assert op.status() == B.MUON_OK
+    dw = max(rel_fro(to_f64(w), wr) for w, wr in zip(W, Wr))
+    dm = max(rel_fro(to_f64(m), mr) for m, mr in zip(M, Mr))
+    print(f"gpt2s free-running drift after {steps} steps: W {dw:.2e}, M {dm:.2e}")
+    assert dw < 5e-2 and dm < 5e-2
+
+
 def test_deterministic_and_resumable():
     wl = I.WORKLOADS["gpt2s"]
     idx = list(range(6))
