@@ -42,7 +42,8 @@ serves as the one primitive; nothing is blocked, fused or reordered.
 Parity pins (tests/test_oracle.py, all CPU):
   * momentum_lerp / nesterov_blend / frobenius_normalize / parameter_write:
     hand-computed worked examples in tests/golden/, special cases
-    (beta = 0, beta = 1, G = M), the textbook Frobenius norm of a 3-4-5 vector.
+    (beta = 0, beta = 1, G = M), the textbook Frobenius norm of a 3-4-5 vector;
+    a zero direction with eps = 0 leaves exactly (1 - lr wd) W.
   * newton_schulz: the cubic (1.5, -0.5, 0) converges to the SVD polar factor
     U V^T; for any (a, b, c) the result equals U diag(phi^k(s_i / (||X||+eps))) V^T
     with phi(x) = a x + b x^3 + c x^5 iterated as a scalar; odd symmetry,
@@ -114,9 +115,18 @@ def frobenius_norm(X) -> float:
 
 
 def frobenius_normalize(X, eps: float) -> np.ndarray:
-    """Step 4: X / (||X||_F + eps).  eps is added to the norm, not to its square."""
+    """Step 4: X / (||X||_F + eps).  eps is added to the norm, not to its square.
+
+    The all-zero matrix has no direction.  For every eps > 0 it normalises to the zero
+    matrix (0 / eps), and with eps = 0 it takes that same value, its limit as eps -> 0+,
+    instead of 0 / 0: a matrix whose momentum direction is exactly zero gets a zero update,
+    so only the weight decay acts on it.
+    """
     X = _f64(X)
-    return X / (frobenius_norm(X) + eps)
+    d = frobenius_norm(X) + eps
+    if d == 0.0:
+        return np.zeros_like(X)
+    return X / d
 
 
 def ns_iteration(X, a: float, b: float, c: float) -> np.ndarray:

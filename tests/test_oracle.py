@@ -236,6 +236,36 @@ def test_zero_input_stays_finite():
     assert np.array_equal(out, np.zeros((8, 16)))
 
 
+def _zero_direction_pin_holds():
+    # A matrix whose gradient and momentum are both zero has U = 0.  With eps = 0 the
+    # normalisation would be 0 / 0; the zero matrix is taken as its own direction (the value it
+    # has for every eps > 0), so O = 0 and the step leaves exactly (1 - lr wd) W.  With the
+    # default eps the same holds without any special case.
+    rng = np.random.default_rng(41)
+    W = rng.standard_normal((6, 10))
+    z = np.zeros_like(W)
+    ok = True
+    for eps in (0.0, 1e-7):
+        hp = O.Hyper(lr=0.05, beta=0.9, weight_decay=0.3, eps=eps, nesterov=True, ns_steps=5)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            W1, M1, O1 = O.muon_step(W, z, z, hp)
+        ok = ok and np.array_equal(O1, z) and np.array_equal(M1, z)
+        ok = ok and np.max(np.abs(W1 - (1.0 - 0.05 * 0.3) * W)) == 0.0
+    return bool(ok)
+
+
+def test_zero_direction_with_zero_eps(monkeypatch):
+    import oracle.muon_oracle as mo
+
+    assert _zero_direction_pin_holds()
+    # a non-zero matrix with eps = 0 is normalised by its norm alone
+    X = np.array([[3.0, 4.0]])
+    assert np.array_equal(O.frobenius_normalize(X, 0.0), np.array([[0.6, 0.8]]))
+    # the unguarded division (0 / 0) turns the zero direction into NaN and fails the pin
+    monkeypatch.setattr(mo, "frobenius_normalize", lambda X, eps: X / (mo.frobenius_norm(X) + eps))
+    assert not _zero_direction_pin_holds()
+
+
 def test_ns_flops_counts():
     # square: 3 m^3 + m^3 per step; wide m x n: 3 m^2 n + m^3
     assert O.ns_flops(1536, 1536, 1) == 4 * 1536 ** 3
