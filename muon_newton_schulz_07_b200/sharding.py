@@ -11,7 +11,8 @@ Ownership is decided by greedy longest-processing-time over the per-matrix
 cost: Newton-Schulz work k (3 m^2 n + m^3) with m = min, n = max, plus a
 bandwidth term for the momentum and parameter passes expressed in the same
 units.  The exchange packs each rank's owned parameters into one contiguous
-buffer and runs one all-gather (NCCL on GPUs, gloo in the CPU tests).
+buffer and runs one all-gather (NCCL on GPUs, gloo in the CPU tests); the
+gradient reduce-scatter sums bf16 gradients in fp32.
 """
 from __future__ import annotations
 
@@ -60,6 +61,12 @@ class ShardedMuon:
     local_step(W_owned, G_owned, M_owned) performs the Muon step on the owned matrices in place
     (by default a MuonStep over their shapes); W, G are the full lists on every rank and M holds
     only the owned momentum buffers, in owned order.
+
+    Data layout of the exchanges: one flat buffer of world segments, segment q holding the
+    matrices rank q owns, back to back in owned order, padded to the longest segment.  Matrix i
+    sits at `offset[i]`.  Packing into and unpacking out of that buffer are multi-tensor copies
+    (one launch each, whatever the number of matrices); a trainer that keeps its gradients in the
+    views returned by gradient_views() skips the packing altogether.
     """
 
     def __init__(self, shapes, rank: int, world: int, local_step: Callable = None, group=None, ns_steps: int = 5,
@@ -70,12 +77,42 @@ class ShardedMuon:
         self.owned = [i for i, r in enumerate(self.owner) if r == rank]
         self.by_rank = [[i for i, r in enumerate(self.owner) if r == q] for q in range(world)]
         self.sizes = [sum(self.shapes[i][0] * self.shapes[i][1] for i in idx) for idx in self.by_rank]
+        self.longest = max(self.sizes) if self.sizes else 0
+        self.offset = [0] * len(self.shapes)
+        for q in range(world):
+            off = q * self.longest
+            for i in self.by_rank[q]:
+                self.offset[i] = off
+                off += self.shapes[i][0] * self.shapes[i][1]
+        self._bufs = {}
         if local_step is None:
             from .optimizer import MuonStep
 
             local_step = MuonStep([self.shapes[i] for i in self.owned], dtype=dtype, device=device)
         self.local_step = local_step
 
+    # ------------------------------------------------------------ flat buffers
+    def _buffer(self, name, numel, dtype, device):
+        """A cached flat buffer, zero-filled when first made (the padding is never written)."""
+        key = (name, dtype, str(device))
+        buf = self._bufs.get(key)
+        if buf is None or buf.numel() != numel:
+            buf = torch.zeros(numel, dtype=dtype, device=device)
+            self._bufs[key] = buf
+        return buf
+
+    def _views(self, flat, idx, base=0):
+        return [flat[self.offset[i] - base:self.offset[i] - base + self.shapes[i][0] * self.shapes[i][1]]
+                .view(self.shapes[i]) for i in idx]
+
+    def gradient_views(self, dtype=torch.bfloat16, device=None):
+        """Views, one per matrix in caller order, into the flat buffer reduce_gradients sends.  A
+        trainer that writes its gradients there (e.g. as the parameters' .grad) sends them without
+        any packing copy."""
+        flat = self._buffer("grad_send", self.world * self.longest, dtype, device)
+        return self._views(flat, range(len(self.shapes)))
+
+    # ------------------------------------------------------------ steps
     def step(self, W, G, M_owned, **hp):
         """A step from gradients already averaged over the ranks (G: the full list on every rank)."""
         if self.owned:
@@ -93,49 +130,43 @@ class ShardedMuon:
     def reduce_gradients(self, G_local):
         """The mean over the ranks of the owned matrices' gradients, in owned order.
 
-        Every rank packs its full list of local gradients into one buffer, rank q's owned matrices
-        in segment q (segments padded to the longest); one reduce-scatter sums segment q onto rank
-        q, which divides by the number of ranks.  The sum runs in the gradients' dtype.  This is
-        the collective that replaces a replicated trainer's all-reduce: each rank receives 1/N of
-        the data instead of all of it.  The returned tensors are views of one fresh buffer.
+        Every rank's gradients sit in the flat send buffer (segment q: the matrices rank q owns);
+        one reduce-scatter sums segment q onto rank q, which divides by the number of ranks and
+        rounds once to the gradients' dtype.  bf16 and fp16 gradients are summed in fp32 (the send
+        buffer is widened by one cast), so the mean carries a single rounding to bf16 instead of
+        one per addition; fp32 and fp64 gradients are summed in their own type.  This is the
+        collective that replaces a replicated trainer's all-reduce: each rank receives 1/N of the
+        data.  The returned tensors are views of one buffer, valid until the next call.
         """
         if self.world == 1:
             return [G_local[i] for i in self.owned]
         ref = G_local[0]
-        longest = max(self.sizes)
-        send = torch.zeros(self.world * longest, dtype=ref.dtype, device=ref.device)
-        for q in range(self.world):
-            off = q * longest
-            for i in self.by_rank[q]:
-                n = G_local[i].numel()
-                send[off:off + n].copy_(G_local[i].reshape(-1))
-                off += n
-        recv = torch.empty(longest, dtype=ref.dtype, device=ref.device)
-        dist.reduce_scatter_tensor(recv, send, op=dist.ReduceOp.SUM, group=self.group)
+        dt, dev = ref.dtype, ref.device
+        send = self._buffer("grad_send", self.world * self.longest, dt, dev)
+        views = self._views(send, range(len(self.shapes)))
+        if any(g.data_ptr() != v.data_ptr() for g, v in zip(G_local, views)):
+            torch._foreach_copy_(views, list(G_local))
+        acc = torch.float32 if dt in (torch.bfloat16, torch.float16) else dt
+        wire = send if acc == dt else self._buffer("grad_wire", send.numel(), acc, dev).copy_(send)
+        recv = self._buffer("grad_recv", self.longest, acc, dev)
+        dist.reduce_scatter_tensor(recv, wire, op=dist.ReduceOp.SUM, group=self.group)
         recv.div_(self.world)
-        out, off = [], 0
-        for i in self.owned:
-            n = G_local[i].numel()
-            out.append(recv[off:off + n].view_as(G_local[i]))
-            off += n
-        return out
+        out = recv if acc == dt else self._buffer("grad_mean", self.longest, dt, dev).copy_(recv)
+        return self._views(out, self.owned, base=self.rank * self.longest)
 
     def exchange(self, W):
-        """Every rank gets the parameters its peers own: one all-gather of packed, padded shards."""
+        """Every rank gets the parameters its peers own: one all-gather of the packed segments
+        (all_gather_into_tensor into the flat layout), unpacked by one multi-tensor copy."""
         if self.world == 1:
             return
         ref = W[0]
-        longest = max(self.sizes)
-        send = torch.zeros(longest, dtype=ref.dtype, device=ref.device)
+        dt, dev = ref.dtype, ref.device
+        send = self._buffer("w_send", self.longest, dt, dev)
         if self.owned:
-            torch.cat([W[i].reshape(-1) for i in self.owned], out=send[: self.sizes[self.rank]])
-        recv = [torch.empty(longest, dtype=ref.dtype, device=ref.device) for _ in range(self.world)]
-        dist.all_gather(recv, send, group=self.group)
-        for q in range(self.world):
-            if q == self.rank:
-                continue
-            off = 0
-            for i in self.by_rank[q]:
-                n = W[i].numel()
-                W[i].copy_(recv[q][off:off + n].view_as(W[i]))
-                off += n
+            torch._foreach_copy_(self._views(send, self.owned, base=self.rank * self.longest),
+                                 [W[i] for i in self.owned])
+        recv = self._buffer("w_recv", self.world * self.longest, dt, dev)
+        dist.all_gather_into_tensor(recv, send, group=self.group)
+        others = [i for i in range(len(self.shapes)) if self.owner[i] != self.rank]
+        if others:
+            torch._foreach_copy_([W[i] for i in others], self._views(recv, others))

@@ -1,7 +1,8 @@
-"""Multi-rank path on CPU: ownership by matrix, and the sharded step (world size 2, gloo).
+"""Multi-rank path on CPU: ownership by matrix, and the sharded step (gloo, world sizes 2 and 4).
 
 The per-rank step is injected: here the float64 oracle steps the owned matrices, so the test checks
 the sharding and the exchange (not the kernels) against the unsharded oracle over the whole set.
+The bf16 gradient mean of the reduce-scatter is bounded element by element for 2 and 4 ranks.
 """
 from __future__ import annotations
 
@@ -135,3 +136,72 @@ def test_reduce_scatter_step_equals_unsharded_step_on_the_mean_gradient():
                 assert np.array_equal(z[f"m{i}"], ref[i][1])
             owned_all += list(z["owned"])
         assert sorted(owned_all) == list(range(len(SHAPES)))
+
+
+# ---------------------------------------------------------------- bf16 gradients: the mean is rounded once
+
+RS_SHAPES = [(64, 96), (96, 64), (128, 128), (32, 256), (8, 8)]
+
+
+def _bf16_local_grads(rank):
+    # heavy-tailed like the GPT-2-small set: N(0, 1e-3^2) with 1 % of the entries x100
+    rng = np.random.default_rng(200 + rank)
+    out = []
+    for s in RS_SHAPES:
+        g = 1e-3 * rng.standard_normal(s)
+        g[rng.random(s) < 0.01] *= 100.0
+        out.append(torch.from_numpy(g).to(torch.bfloat16))
+    return out
+
+
+def _worker_bf16_mean(rank, world, port, outdir):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        sh = ShardedMuon(RS_SHAPES, rank, world, local_step=lambda *a, **k: None)
+        G = _bf16_local_grads(rank)
+        got = sh.reduce_gradients(G)
+        first = [g.to(torch.float64).numpy().copy() for g in got]
+        # the same gradients written straight into the send buffer's views: no packing copy, same mean
+        views = sh.gradient_views(torch.bfloat16)
+        for v, g in zip(views, G):
+            v.copy_(g)
+        again = sh.reduce_gradients(views)
+        for a, b in zip(first, again):
+            assert np.array_equal(a, b.to(torch.float64).numpy())
+        np.savez(os.path.join(outdir, f"rank{rank}.npz"), owned=np.array(sh.owned),
+                 **{f"g{i}": a for i, a in zip(sh.owned, first)})
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_bf16_gradient_mean_is_rounded_once(world):
+    # The reduce-scatter sums bf16 gradients in fp32 and rounds the mean to bf16 once, so every
+    # element lies within half a bf16 spacing of the exact mean of the ranks' bf16 values (plus
+    # the fp32 summation, a few 2^-24 of the summands).  Summing in bf16 instead would round after
+    # every addition; with two ranks that is still one rounding, with four ranks it breaks this
+    # bound by orders of magnitude where a spike (x100) meets small values (printed).
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_worker_bf16_mean, args=(world, _free_port(), d), nprocs=world, join=True,
+                           start_method="spawn")
+        locals_ = [[g.to(torch.float64).numpy() for g in _bf16_local_grads(r)] for r in range(world)]
+        exact = [sum(gs) / world for gs in zip(*locals_)]
+        mag = [sum(np.abs(g) for g in gs) / world for gs in zip(*locals_)]
+        seen = []
+        worst_bf16_sum = 0.0
+        for r in range(world):
+            z = np.load(os.path.join(d, f"rank{r}.npz"))
+            for i in z["owned"]:
+                got = z[f"g{i}"]
+                half = 0.5 * np.exp2(np.floor(np.log2(np.maximum(np.abs(exact[i]), 1e-37))) - 7)
+                bound = half + 2.0 ** -21 * mag[i]
+                assert np.all(np.abs(got - exact[i]) <= bound), (world, i)
+                # the same mean accumulated in bf16, for the record
+                acc = torch.zeros(RS_SHAPES[i], dtype=torch.bfloat16)
+                for g in (torch.from_numpy(l[i]).to(torch.bfloat16) for l in locals_):
+                    acc = acc + g
+                bsum = (acc / world).to(torch.float64).numpy()
+                worst_bf16_sum = max(worst_bf16_sum, float(np.max(np.abs(bsum - exact[i]) / np.maximum(bound, 1e-30))))
+                seen.append(int(i))
+        assert sorted(seen) == list(range(len(RS_SHAPES)))
+        print(f"world {world}: bf16 accumulation would reach {worst_bf16_sum:.2f} x the fp32-accumulation bound")
