@@ -44,10 +44,15 @@ def parse():
                          "split one set by matrix and all-gather the parameters (strong scaling)")
     ap.add_argument("--matrices", type=int, default=0,
                     help="use only the first N matrices of the workload (profiling captures of a smaller case)")
+    ap.add_argument("--schedule", choices=["auto", "staged", "fused"], default="auto",
+                    help="Newton-Schulz launch schedule of the library (staged: one launch per stage)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW leg (non-matrix parameters)")
     ap.add_argument("--reference-budget-s", type=float, default=150.0)
+    ap.add_argument("--extra", default=",".join(EXTRA_LEGS),
+                    help="further workloads timed after the d24 headline on one GPU (comma list of "
+                         + ", ".join(EXTRA_LEGS) + "; empty to skip)")
     return ap.parse_args()
 
 
@@ -252,8 +257,14 @@ def run_reference(args, rank):
               f"{', '.join(f'{r}x{c}' for r, c in shapes)}; the full-set step time is the sum over shapes of "
               f"count x median time (extrapolated)")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": done,
-        "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "ms_per_step_is_estimate": True,
+        "timed": {"unit": "one single-matrix oracle step (one matrix of one distinct shape)",
+                  "count": done, "per_shape_median_s": {f"{r}x{c}": statistics.median(times[(r, c)])
+                                                        for r, c in shapes},
+                  "full_step_estimate": "sum over shapes of matrix count x median single-matrix time"},
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "matrices": len(wl.shapes), "params": I.param_count(wl),
                    "ns_steps": args.ns_steps},
@@ -264,6 +275,204 @@ def run_reference(args, rank):
 
 
 # ---------------------------------------------------------------- the Muon arm
+
+NS_KINDS = ("gram", "poly", "update", "ns_small", "ns_fused")
+# Targets for the two kinds of kernel: the Newton-Schulz products at >= 60 % of the dense bf16
+# tensor peak, the momentum/norm pass at >= 80 % of the HBM copy bandwidth.
+TARGET_NS_FRAC = 0.60
+TARGET_MOMENTUM_FRAC = 0.80
+
+
+def kernel_table(prof, shapes, k, elem, steps, peaks, peak_src, wl_name):
+    """Per-kernel times from the library's event tracing, turned into rates against the peaks.
+
+    The headline fraction of a tensor-core kernel is taken against the burst bf16 peak (the
+    kernels run near the maximum clock inside a step of tens of milliseconds); the fraction of the
+    sustained (power-capped) peak is given beside it.
+    """
+    fl = flops_by_kind(shapes, k)
+    by = bytes_by_kind(shapes, elem)
+    kern = {kname: {"ms_total": ms, "launches": cnt, "ms_per_launch": (ms / cnt if cnt else None)}
+            for kname, (ms, cnt) in prof.items() if cnt}
+    per_launch_units = {
+        "gram": fl["gram"] / k if k else 0, "poly": fl["poly"] / k if k else 0,
+        "update": fl["update"] / k if k else 0,
+        "momentum_norm": by["momentum_norm"], "write": by["write"],
+        "ns_small": sum(fl.values()),  # one launch runs every iteration of the step
+        "ns_fused": sum(fl.values()),
+    }
+    for kname, kd in kern.items():
+        if kname in NS_KINDS:
+            kd["tflops"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e12
+            kd["frac_of_burst_peak"] = kd["tflops"] / peaks["bf16_tflops"]
+            kd["frac_of_sustained_peak"] = kd["tflops"] / peaks["bf16_tflops_sustained"]
+        elif kname in ("momentum_norm", "write"):
+            kd["gbs"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e9
+            kd["frac_of_hbm"] = kd["gbs"] / peaks["hbm_gbs"]
+    dominant = max(kern, key=lambda x: kern[x]["ms_total"])
+    if dominant in NS_KINDS:
+        ach = kern[dominant]["tflops"]
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], "traffic": measured_traffic(dominant, wl_name),
+                "kernel": {"ns_small": "ns_small_kernel", "ns_fused": "ns_fused_kernel (every iteration)"}.get(
+                    dominant, f"ns_gemm_tc_kernel ({dominant})"),
+                "peak_source": f"{peak_src} bf16_tflops (burst, dense)",
+                "frac_sustained": ach / peaks["bf16_tflops_sustained"],
+                "peak_sustained": peaks["bf16_tflops_sustained"]}
+    else:
+        ach = kern[dominant]["gbs"]
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": None, "kernel": dominant,
+                "peak_source": f"{peak_src} hbm_gbs"}
+    ns_ms = sum(kern[x]["ms_total"] for x in NS_KINDS if x in kern) / steps
+    ns_flops = sum(fl.values())
+    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms > 0 else None
+    ns = {"tflops": ns_tflops,
+          "frac_of_burst_peak": (ns_tflops / peaks["bf16_tflops"]) if ns_tflops else None,
+          "frac_of_sustained_peak": (ns_tflops / peaks["bf16_tflops_sustained"]) if ns_tflops else None,
+          "ms_per_step": ns_ms, "flops_per_step": ns_flops}
+    targets = {"ns_frac_of_burst_peak": {"value": ns["frac_of_burst_peak"], "target": TARGET_NS_FRAC,
+                                         "met": bool(ns_tflops and ns["frac_of_burst_peak"] >= TARGET_NS_FRAC)}}
+    if "momentum_norm" in kern:
+        f = kern["momentum_norm"]["frac_of_hbm"]
+        targets["momentum_norm_frac_of_hbm"] = {"value": f, "target": TARGET_MOMENTUM_FRAC,
+                                                "met": bool(f >= TARGET_MOMENTUM_FRAC)}
+    return kern, roof, ns, targets
+
+
+def make_inputs(wl, dev, dt, rank, shapes=None):
+    """W, M and two gradient sets of a workload on the device (seeded; every rank its own G)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    from muon_newton_schulz_07_b200 import inputs as I
+
+    n = len(shapes if shapes is not None else wl.shapes)
+
+    def to_dev(a):
+        return torch_from(a, dev, dt)
+
+    def gen(fn):
+        with ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
+            return [to_dev(a) for a in ex.map(fn, range(n))]
+
+    W = gen(lambda i: I.weight(wl, i))
+    if wl.name.startswith("stress"):
+        # P diag(s) Q^T drawn on the device (host QR of the whole set takes minutes); G = M
+        import torch
+
+        M = [I.stress_momentum_torch(wl, i, dev).to(dt) for i in range(n)]
+        G_sets = [[m.clone() for m in M] for _ in range(2)]
+        torch.cuda.synchronize(dev)
+        return W, M, G_sets
+    M = gen(lambda i: I.momentum(wl, i))
+    G_sets = [gen(lambda i, s=s: I.gradient(wl, 1 + s + 1000 * rank, i)) for s in range(2)]
+    return W, M, G_sets
+
+
+def torch_from(a, dev, dt):
+    import torch
+
+    return torch.from_numpy(a).to(dev).to(dt)
+
+
+def timed_steps(step_fn, G_sets, steps, warmup, op, dev, stream, local_rank, sync_all, in_bytes, B):
+    """W warm-up steps, then `steps` timed steps with CUDA events on the launching stream and the
+    library's per-kernel tracing; clocks sampled meanwhile.  Inputs smaller than L2 get a 512 MB
+    scratch write before every timed step (outside that step's events)."""
+    import torch
+
+    for i in range(warmup):
+        step_fn(G_sets[i % 2])
+    sync_all()
+    if op.status() != B.MUON_OK:
+        raise RuntimeError("device status after warm-up is not OK")
+    clocks = ClockSampler(gpu_index_for(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if in_bytes < L2_FLUSH_BELOW else None
+    B.muon_profile_begin(op.handle, steps)
+    sync_all()
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            step_fn(G_sets[i % 2])
+        e1.record(stream)
+        sync_all()
+        ms_total = e0.elapsed_time(e1)
+    else:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step_fn(G_sets[i % 2])
+            ev[i][1].record(stream)
+        sync_all()
+        ms_total = sum(a.elapsed_time(b) for a, b in ev)
+    clk = clocks.stop()
+    prof = B.muon_profile_end(op.handle)
+    status = op.status()
+    if status != B.MUON_OK:
+        raise RuntimeError(f"device status after the timed steps: {B.STATUS.get(status, status)}")
+    return ms_total, prof, clk, flush is not None
+
+
+# Further workloads timed after the headline one (one GPU only), each its own block of the line.
+EXTRA_LEGS = {
+    "l38b": ("l38b", 5, 10),      # (workload, Newton-Schulz steps, timed steps)
+    "stress_k5": ("stress", 5, 20),
+    "stress_k10": ("stress", 10, 10),
+    "gpt2s": ("gpt2s", 5, 50),
+}
+
+
+def run_extra_leg(leg, warmup, dev, local_rank, peaks, peak_src, schedule="auto", cache=None):
+    """One further workload leg; `cache` keeps the last workload's inputs for the next leg."""
+    import torch
+
+    from muon_newton_schulz_07_b200 import binding as B
+    from muon_newton_schulz_07_b200 import inputs as I
+    from muon_newton_schulz_07_b200.optimizer import MuonStep
+
+    name, k, steps = EXTRA_LEGS[leg]
+    wl = I.WORKLOADS[name]
+    shapes = list(wl.shapes)
+    dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    t0 = time.perf_counter()
+    if cache is not None and cache.get("name") == name:
+        W, M, G_sets = cache["inputs"]
+    else:
+        if cache is not None:
+            cache.clear()
+            torch.cuda.empty_cache()
+        W, M, G_sets = make_inputs(wl, dev, dt, 0)
+        if cache is not None:
+            cache.update(name=name, inputs=(W, M, G_sets))
+    gen_s = time.perf_counter() - t0
+    op = MuonStep(shapes, dtype=dt, device=dev, schedule=schedule)
+    stream = torch.cuda.current_stream(dev)
+
+    def step_fn(Gs):
+        op(W, Gs, M, ns_steps=k)
+
+    in_bytes = sum(t.numel() * t.element_size() for t in list(W) + list(M) + list(G_sets[0]))
+    ms_total, prof, clk, flushed = timed_steps(step_fn, G_sets, steps, warmup, op, dev, stream, local_rank,
+                                               lambda: torch.cuda.synchronize(dev), in_bytes, B)
+    kern, roof, ns, targets = kernel_table(prof, shapes, k, 4 if dt == torch.float32 else 2, steps, peaks, peak_src,
+                                           wl.name)
+    ms = ms_total / steps
+    out = {"workload": wl.name, "ns_steps": k, "matrices": len(shapes), "params": I.param_count(wl),
+           "steps": steps, "warmup": warmup, "ms_per_step": ms, "value": 1000.0 / ms, "unit": UNIT,
+           "roofline": roof, "ns": ns, "kernels": kern, "targets": targets,
+           "gpu_launches": op.launches_per_step(k) * steps, "clocks": clk,
+           "l2": "flushed before every timed step" if flushed else "inputs larger than L2, no flush",
+           "input_generation_s": gen_s}
+    op.close()
+    del W, M, G_sets
+    if cache is None:
+        torch.cuda.empty_cache()
+    return out
+
 
 def run_muon(args, rank, world, local_rank):
     import numpy as np
@@ -289,33 +498,22 @@ def run_muon(args, rank, world, local_rank):
     k = args.ns_steps
     dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
 
-    def to_dev(a):
-        return torch.from_numpy(a).to(dev).to(dt)
-
     # Every rank steps its own parameter set; gradients differ by rank through the step seed.
-    from concurrent.futures import ThreadPoolExecutor
-
-    def gen(fn):
-        with ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
-            return [to_dev(a) for a in ex.map(fn, range(n))]
-
-    W = gen(lambda i: I.weight(wl, i))
-    M = gen(lambda i: I.momentum(wl, i))
-    G_sets = [gen(lambda i, s=s: I.gradient(wl, 1 + s + 1000 * rank, i)) for s in range(2)]
+    W, M, G_sets = make_inputs(wl, dev, dt, rank, shapes)
     sharded = args.mode == "sharded" and world > 1
     if sharded:
         # strong scaling: each rank owns a share of the matrices, steps only those and all-gathers W
         from muon_newton_schulz_07_b200.sharding import ShardedMuon
 
         probe = ShardedMuon(shapes, rank, world, local_step=lambda *a, **kw: None, ns_steps=k)
-        op = MuonStep([shapes[i] for i in probe.owned], dtype=dt, device=dev)
+        op = MuonStep([shapes[i] for i in probe.owned], dtype=dt, device=dev, schedule=args.schedule)
         sh = ShardedMuon(shapes, rank, world, local_step=op, ns_steps=k)
         M_owned = [M[i] for i in sh.owned]
 
         def step_fn(Gs):
             sh.step(W, Gs, M_owned, ns_steps=k)
     else:
-        op = MuonStep(shapes, dtype=dt, device=dev)
+        op = MuonStep(shapes, dtype=dt, device=dev, schedule=args.schedule)
 
         def step_fn(Gs):
             op(W, Gs, M, ns_steps=k)
@@ -334,43 +532,9 @@ def run_muon(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    for i in range(args.warmup):
-        step_fn(G_sets[i % 2])
-    sync_all()
-    if op.status() != B.MUON_OK:
-        raise RuntimeError("device status after warm-up is not OK")
-
-    clocks = ClockSampler(gpu_index_for(local_rank))
-    clocks.start()
-    time.sleep(0.3)
-    # Inputs smaller than the L2 cache would stay resident between steps: then a scratch buffer
-    # larger than L2 is written before every timed step, outside that step's own events.
     in_bytes = sum(t.numel() * t.element_size() for t in list(W) + list(M) + list(G_sets[0]))
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if in_bytes < L2_FLUSH_BELOW else None
-    B.muon_profile_begin(op.handle, args.steps)
-    sync_all()
-    if flush is None:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(args.steps):
-            step_fn(G_sets[i % 2])
-        e1.record(stream)
-        sync_all()
-        ms_total = e0.elapsed_time(e1)
-    else:
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record(stream)
-            step_fn(G_sets[i % 2])
-            ev[i][1].record(stream)
-        sync_all()
-        ms_total = sum(a.elapsed_time(b) for a, b in ev)
-    clk = clocks.stop()
-    prof = B.muon_profile_end(op.handle)
-    status = op.status()
-    if status != B.MUON_OK:
-        raise RuntimeError(f"device status after the timed steps: {B.STATUS.get(status, status)}")
+    ms_total, prof, clk, flushed = timed_steps(step_fn, G_sets, args.steps, args.warmup, op, dev, stream, local_rank,
+                                               sync_all, in_bytes, B)
     ms_per_step = max_over_ranks(ms_total / args.steps)
     value = (1 if sharded else world) * 1000.0 / ms_per_step
 
@@ -411,53 +575,30 @@ def run_muon(args, rank, world, local_rank):
                "d2h_bytes_per_step": 4 * len(op.shapes), "ms_per_step": e2e_ms, "steps": ksteps,
                "path": ("pinned host G -> device copy, then the sharded step" if sharded else
                         "pinned host G -> device copy on a side stream overlapping the previous step "
-                        "(MuonStep.step_from_host -> C ABI muon_step), norms -> pinned host")}
+                        "(MuonStep.step_from_host -> C ABI muon_step), per-matrix norms -> pinned host; "
+                        "W and M stay resident on the device (an optimizer's state lives there), so "
+                        "they are not copied back")}
 
     # ------------------------------------------------------------ roofline
     peaks, peak_src = load_peaks()
-    fl = flops_by_kind(shapes, k)
-    by = bytes_by_kind(shapes, 4 if dt == torch.float32 else 2)
-    kern = {kname: {"ms_total": ms, "launches": cnt, "ms_per_launch": (ms / cnt if cnt else None)}
-            for kname, (ms, cnt) in prof.items() if cnt}
-    dominant = max(kern, key=lambda x: kern[x]["ms_total"])
-    per_launch_units = {
-        "gram": fl["gram"] / k, "poly": fl["poly"] / k, "update": fl["update"] / k,
-        "momentum_norm": by["momentum_norm"], "write": by["write"],
-        "ns_small": sum(fl.values()),  # one launch runs every iteration of the step
-    }
-    if dominant in ("gram", "poly", "update", "ns_small"):
-        ach = per_launch_units[dominant] / (kern[dominant]["ms_per_launch"] * 1e-3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                "traffic": measured_traffic(dominant, wl.name), "kernel": f"ns_gemm_tc_kernel ({dominant})",
-                "peak_source": f"{peak_src} bf16_tflops_sustained"}
-    else:
-        ach = per_launch_units[dominant] / (kern[dominant]["ms_per_launch"] * 1e-3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                "traffic": None, "kernel": dominant, "peak_source": f"{peak_src} hbm_gbs"}
-    ns_ms = sum(kern[x]["ms_total"] for x in ("gram", "poly", "update", "ns_small") if x in kern) / args.steps
-    ns_flops = sum(fl.values())
-    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms > 0 else None
-    for kname, kd in kern.items():
-        if kname in ("gram", "poly", "update", "ns_small"):
-            kd["tflops"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e12
-            kd["frac_of_sustained_peak"] = kd["tflops"] / peaks["bf16_tflops_sustained"]
-        elif kname in ("momentum_norm", "write"):
-            kd["gbs"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e9
-            kd["frac_of_hbm"] = kd["gbs"] / peaks["hbm_gbs"]
+    kern, roof, ns, targets = kernel_table(prof, shapes, k, 4 if dt == torch.float32 else 2, args.steps, peaks,
+                                           peak_src, wl.name)
 
     # ------------------------------------------------------------ AdamW leg (the non-matrix half)
     adamw = None
     if not args.no_adamw and wl.name == "d24":
+        from concurrent.futures import ThreadPoolExecutor
+
         from muon_newton_schulz_07_b200.optimizer import adamw_step
 
         sizes = I.D24_ADAMW_SIZES
         with ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
-            P = [to_dev(a) for a in ex.map(lambda i: I.adamw_param(0, i, I.TID_W, sizes[i]), range(len(sizes)))]
-            Gd = [to_dev(a) for a in ex.map(lambda i: I.adamw_param(1, i, I.TID_G, sizes[i]), range(len(sizes)))]
-        Ma = [torch.zeros(n, dtype=torch.float32, device=dev) for n in sizes]
-        Va = [torch.zeros(n, dtype=torch.float32, device=dev) for n in sizes]
+            P = [torch_from(a, dev, dt) for a in ex.map(lambda i: I.adamw_param(0, i, I.TID_W, sizes[i]),
+                                                        range(len(sizes)))]
+            Gd = [torch_from(a, dev, dt) for a in ex.map(lambda i: I.adamw_param(1, i, I.TID_G, sizes[i]),
+                                                         range(len(sizes)))]
+        Ma = [torch.zeros(n_, dtype=torch.float32, device=dev) for n_ in sizes]
+        Va = [torch.zeros(n_, dtype=torch.float32, device=dev) for n_ in sizes]
         for i in range(args.warmup):
             adamw_step(P, Gd, Ma, Va, i + 1, lr=3e-3, betas=(0.8, 0.95), eps=1e-10, weight_decay=0.0)
         sync_all()
@@ -471,7 +612,7 @@ def run_muon(args, rank, world, local_rank):
         nel = sum(sizes)
         a_bytes = nel * (2 + 2 + 2 + 8 + 8)  # p read+write, g read, m and v read+write (fp32)
         a_gbs = a_bytes / (a_ms * 1e-3) / 1e9
-        adamw = {"params": nel, "ms_per_step": a_ms, "gbs": a_gbs, "frac_of_hbm": a_gbs / load_peaks()[0]["hbm_gbs"],
+        adamw = {"params": nel, "ms_per_step": a_ms, "gbs": a_gbs, "frac_of_hbm": a_gbs / peaks["hbm_gbs"],
                  "bytes_per_step": a_bytes, "launches_per_step": 1,
                  "set": "d24 non-matrix parameters: 14 x 32768x1536 tables + 48 scalars, bf16, fp32 moments"}
         del P, Gd, Ma, Va
@@ -481,6 +622,19 @@ def run_muon(args, rank, world, local_rank):
         step_s, sample = oracle_sample(wl)
         cpu = {"value": 1.0 / step_s, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample}
 
+    # ------------------------------------------------------------ further workloads (one GPU only)
+    extra = None
+    if world == 1 and args.extra and wl.name == "d24" and not args.matrices:
+        op.close()
+        del W, M, G_sets
+        torch.cuda.empty_cache()
+        extra = {}
+        cache = {}
+        for leg in [x for x in args.extra.split(",") if x]:
+            extra[leg] = run_extra_leg(leg, args.warmup, dev, local_rank, peaks, peak_src, args.schedule, cache)
+        cache.clear()
+        torch.cuda.empty_cache()
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -488,18 +642,17 @@ def run_muon(args, rank, world, local_rank):
             "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "matrices": n, "params": I.param_count(wl), "ns_steps": k,
-                       "groups": op.n_groups,
+                       "groups": op.n_groups, "schedule": args.schedule,
                        "parallelism": (f"sharded by matrix over {world} ranks + all-gather of W (NCCL)" if sharded
                                        else f"replica x{world} (one parameter set per GPU)"),
                        "l2": ("inputs larger than L2 (W, G, M: %.2f GB per GPU), no flush" % (in_bytes / 1e9)
-                              if flush is None else
+                              if not flushed else
                               "inputs smaller than L2 (W, G, M: %.1f MB): a 512 MB buffer is written before every "
                               "timed step, outside the step's events" % (in_bytes / 1e6)),
                        "description": wl.description},
             "roofline": roof,
-            "ns": {"tflops": ns_tflops, "frac_of_sustained_peak": (ns_tflops / peaks["bf16_tflops_sustained"])
-                   if ns_tflops else None, "frac_of_burst_peak": (ns_tflops / peaks["bf16_tflops"])
-                   if ns_tflops else None, "ms_per_step": ns_ms, "flops_per_step": ns_flops},
+            "ns": ns,
+            "targets": targets,
             "kernels": kern,
             "cpu_baseline": cpu,
             "adamw": adamw,
@@ -507,8 +660,11 @@ def run_muon(args, rank, world, local_rank):
             "gpu_launches": launches * args.steps,
             "clocks": clk,
         }
+        if extra is not None:
+            line["workloads"] = extra
         print(json.dumps(line), flush=True)
-    op.close()
+    if extra is None:
+        op.close()
 
 
 def main():

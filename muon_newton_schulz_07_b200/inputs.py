@@ -89,6 +89,34 @@ def stress_factors(wid, idx, rows, cols):
     return P, s, Q
 
 
+def stress_momentum_torch(wl: Workload, idx: int, device):
+    """The stress set's matrix idx made on `device` with torch (same recipe, another stream).
+
+    M = P diag(s) Q^T with P, Q the orthonormal factors of torch.linalg.qr of Gaussian matrices
+    drawn by torch's generator (seeded from the same (workload, matrix, tensor) seeds), columns'
+    signs fixed by diag(R), and s log-uniform in [1e-6, 1] (NumPy, as in stress_factors).  The
+    values differ from momentum() (another random stream and QR), the structure does not.  QR of
+    the 256 matrices on the host takes minutes; on a GPU it takes seconds, so the full-size GPU
+    runs (tests and benchmark legs) draw the stress set here.  Returns a float32 tensor.
+    """
+    import torch
+
+    r, c = wl.shapes[idx]
+    k = min(r, c)
+
+    def factor(n, tid):
+        seed = int(np.random.SeedSequence([wl.wid, 0, idx, tid]).generate_state(1)[0])
+        gen = torch.Generator(device=device).manual_seed(seed)
+        a = torch.randn((n, k), generator=gen, device=device, dtype=torch.float64)
+        q, rr = torch.linalg.qr(a)
+        return q * torch.sign(torch.diagonal(rr))
+
+    P, Q = factor(r, TID_P), factor(c, TID_Q)
+    sv = np.exp(rng_for(wl.wid, 0, idx, TID_S).uniform(np.log(1e-6), 0.0, k))
+    s = torch.from_numpy(sv).to(device)
+    return ((P * s) @ Q.T).to(torch.float32)
+
+
 def weight(wl: Workload, idx: int) -> np.ndarray:
     r, c = wl.shapes[idx]
     if wl.name == "single256":

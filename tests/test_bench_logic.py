@@ -65,7 +65,10 @@ def test_reference_arm_times_every_shape_even_on_short_runs(monkeypatch, capsys)
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     shapes = sorted(set(I.WORKLOADS["d24"].shapes))
     assert sorted(set(calls)) == shapes           # every distinct shape was stepped
-    assert line["steps"] >= len(shapes) and line["impl"] == "reference"
+    # the line reports the requested steps, and separately how many single-matrix timings it took
+    assert line["steps"] == 1 and line["impl"] == "reference"
+    assert line["timed"]["count"] >= len(shapes) and line["ms_per_step_is_estimate"] is True
+    assert sorted(line["timed"]["per_shape_median_s"]) == sorted(f"{r}x{c}" for r, c in shapes)
     assert line["value"] > 0 and np.isfinite(line["value"])
     assert line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0
@@ -75,3 +78,21 @@ def test_reference_arm_is_silent_on_other_ranks(capsys):
     args = argparse.Namespace(workload="d24", steps=1, warmup=1, ns_steps=5, gpus=2, reference_budget_s=1.0)
     bench.run_reference(args, rank=1)
     assert capsys.readouterr().out == ""
+
+
+def test_kernel_table_uses_the_burst_peak_for_the_headline():
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    shapes = [(1536, 1536)] * 4
+    k = 5
+    fl = bench.flops_by_kind(shapes, k)
+    # every Update launch takes 1 ms, the other kernels less
+    prof = {"momentum_norm": (0.1 * 2, 2), "gram": (0.2 * 2 * k, 2 * k), "poly": (0.1 * 2 * k, 2 * k),
+            "update": (1.0 * 2 * k, 2 * k), "write": (0.0, 0), "sgemm_ref": (0.0, 0), "ns_small": (0.0, 0)}
+    kern, roof, ns, targets = bench.kernel_table(prof, shapes, k, 2, 2, peaks, "measured", "d24")
+    upd = fl["update"] / k / 1e-3 / 1e12
+    assert roof["kernel"].endswith("(update)") and abs(roof["achieved"] - upd) < 1e-9
+    assert abs(roof["frac"] - upd / 1600.0) < 1e-12 and abs(roof["frac_sustained"] - upd / 1400.0) < 1e-12
+    assert abs(kern["gram"]["frac_of_burst_peak"] - kern["gram"]["tflops"] / 1600.0) < 1e-12
+    assert "write" not in kern
+    assert set(targets) == {"ns_frac_of_burst_peak", "momentum_norm_frac_of_hbm"}
+    assert targets["momentum_norm_frac_of_hbm"]["met"] == (kern["momentum_norm"]["frac_of_hbm"] >= 0.80)

@@ -71,3 +71,23 @@ def test_stress_structure(idx):
     assert np.array_equal(I.gradient(wl, 1, idx), M)  # G = M, so the Nesterov blend is M
     sv = np.linalg.svd(M.astype(np.float64), compute_uv=False)
     assert np.allclose(np.sort(sv)[::-1][:8], np.sort(s)[::-1][:8], rtol=1e-5)
+
+
+@pytest.mark.parametrize("idx", [0, 64, 128, 192])
+def test_stress_structure_torch_generator(idx):
+    # the device-side generator (used by the full-size GPU runs) follows the same recipe; run on
+    # the CPU here: orthonormal factors, singular values exactly the log-uniform s
+    import torch
+
+    wl = I.WORKLOADS["stress"]
+    r, c = wl.shapes[idx]
+    M = I.stress_momentum_torch(wl, idx, "cpu")
+    assert M.shape == (r, c) and M.dtype == torch.float32
+    _, s, _ = I.stress_factors(wl.wid, idx, r, c)
+    sv = np.linalg.svd(M.double().numpy(), compute_uv=False)
+    big = np.sort(s)[::-1]
+    # fp32 storage: the largest singular values match to fp32 accuracy
+    assert np.allclose(sv[:16], big[:16], rtol=1e-5)
+    # same seeds, same matrix; another matrix differs
+    assert torch.equal(M, I.stress_momentum_torch(wl, idx, "cpu"))
+    assert not torch.equal(M[:8, :8], I.stress_momentum_torch(wl, idx + 1, "cpu")[:8, :8])
