@@ -2,8 +2,9 @@
 
 The oracle cannot step 144-168 matrices of these sizes in seconds, so it checks sampled matrices:
 the first, middle and last matrix of each distinct shape.  M1 and W1 come from the caller's
-tensors; the orthogonalised direction from a second step with W = 0.  The conditioning-stress set is checked against the scalar polynomial, singular
-value by singular value.
+tensors (element by element); the orthogonalised direction from a second step with W = 0.  The
+whole conditioning-stress set runs through one handle and three matrices of each shape are
+checked against the scalar polynomial, singular value by singular value.
 """
 from __future__ import annotations
 
@@ -19,7 +20,7 @@ from muon_newton_schulz_07_b200 import binding as B
 from muon_newton_schulz_07_b200 import inputs as I
 from muon_newton_schulz_07_b200.optimizer import MuonStep
 
-from helpers import bf16_ulp, rel_fro, to_f64
+from helpers import assert_m1_elementwise, assert_w1_elementwise, bf16_ulp, rel_fro, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -71,42 +72,74 @@ def test_full_set_step_sampled(name):
         assert torch.equal(M[i], Mz[i])
         bound = 0.5 * 1.01 * np.linalg.norm(bf16_ulp(W1r)) + 0.02 * O.shape_scale(r, c) * 2e-2 * np.linalg.norm(Or)
         assert np.linalg.norm(to_f64(W[i]) - W1r) <= bound, (name, i)
+        assert_m1_elementwise(to_f64(M[i]), M1r, M0, G0, torch.bfloat16, what=f"M1 {name} {i}")
+        Wzr = O.parameter_write(np.zeros_like(W0), Or, 0.02, 0.0)
+        assert_w1_elementwise(to_f64(W[i]), W1r, to_f64(Wz[i]), Wzr, W0, torch.bfloat16, what=f"W1 {name} {i}")
     print(f"{name}: {len(check)} sampled matrices, worst O error {worst:.3e}")
     op.close()
 
 
-STRESS_IDX = [0, 1, 64, 65, 128, 129, 192, 193]  # two matrices of each stress shape, full size
+# The whole stress set (256 matrices, three shape groups: 512 x 4096 with its transpose, 2048^2,
+# 8192 x 1024) goes through one handle; three matrices of each shape are checked.
+STRESS_SAMPLE = [0, 31, 63, 64, 95, 127, 128, 159, 191, 192, 223, 255]
 
 # Largest value of the quintic on [0, 1]: normalised singular values start in [0, 1] and
 # the iteration keeps them in [0, PHI_MAX] (the polynomial has no real root there).
 PHI_MAX = 1.2024
 
 
-def linear_gain(x, k, abc=O.QUINTIC):
-    """|d phi^k / dx| along the scalar trajectory (chain rule)."""
+def propagated_gain(x, k, abc=O.QUINTIC):
+    """First-order amplification of the roundings along the scalar trajectory of x.
+
+    Every iteration stores X (and A, B') rounded, so a perturbation enters before each step j and
+    is amplified by the derivatives of the steps that follow it only: sum over j of
+    prod_{t >= j} |phi'(x_t)|.  The product over the whole trajectory alone (j = 0) understates it
+    when the trajectory passes near the critical point of phi (x = 0.5545, phi' = 0, where phi
+    reaches 1.2024): the factor there is tiny, yet roundings made after it are amplified by
+    |phi'(1.2024)| = 3.97 and the steps after.
+    """
     a, b, c = abc
-    g = np.ones_like(x)
+    d = []
     for _ in range(k):
-        g = g * np.abs(a + 3 * b * x * x + 5 * c * x ** 4)
+        d.append(np.abs(a + 3 * b * x * x + 5 * c * x ** 4))
         x = a * x + b * x ** 3 + c * x ** 5
+    g = np.zeros_like(x)
+    suffix = np.ones_like(x)
+    for j in reversed(range(k)):
+        suffix = suffix * d[j]
+        g = g + suffix
     return g
 
 
+_STRESS = {}
+
+
+def stress_inputs():
+    """The stress set's momenta as fp32 device tensors (drawn on the device by the input module's
+    torch generator: same recipe as the NumPy one, whose host QR of 256 matrices takes minutes),
+    generated once per test session."""
+    if "X" not in _STRESS:
+        wl = I.WORKLOADS["stress"]
+        _STRESS["X"] = [I.stress_momentum_torch(wl, i, "cuda") for i in range(len(wl.shapes))]
+    return I.WORKLOADS["stress"].shapes, _STRESS["X"]
+
+
 def stress_run(mode, dtype, k):
-    wl = I.WORKLOADS["stress"]
-    shapes = [wl.shapes[i] for i in STRESS_IDX]
-    X = [torch.from_numpy(I.momentum(wl, i)).cuda().to(dtype) for i in STRESS_IDX]
+    shapes, X32 = stress_inputs()
+    X = [x.to(dtype) for x in X32]
     Os = [torch.empty_like(x) for x in X]
     op = MuonStep(shapes, dtype=dtype, mode=mode)
+    assert op.n_groups == 3
     op.orthogonalize(X, Os, ns_steps=k)
     torch.cuda.synchronize()
     assert op.status() == B.MUON_OK
     op.close()
-    for x, o, s in zip(X, Os, shapes):
-        U = to_f64(x)
+    for i in STRESS_SAMPLE:
+        U = to_f64(X[i])
         P, sv, Qt = np.linalg.svd(U, full_matrices=False)
         xs = sv / (math.sqrt(float(np.sum(sv * sv))) + 1e-7)
-        yield s, U, to_f64(o), P, xs, Qt
+        yield shapes[i], U, to_f64(Os[i]), P, xs, Qt
+    del X, Os
 
 
 @pytest.mark.parametrize("k", [5, 10])
@@ -115,11 +148,14 @@ def test_stress_fp32_reference_mode(k):
     # D = P^T O Q (SVD of the input, fp64) is diagonal with the scalar polynomial's values.
     # After 10 steps the smallest directions are amplified by up to a^10 = 2.35e5, so one
     # fp32 rounding (u = 2^-24) of X can move them by ~1e-2: there, as for the bf16 path,
-    # the directions with gain * u <= 1e-2 are held to 1e-4 and all of O to the band.
+    # the directions with propagated gain * u <= 1e-2 are held to 1e-4 and all of O to the
+    # band.  The whole-matrix error is printed (the design notes record it).
     u = 2.0 ** -24
+    worst_whole = 0.0
     for s, U, Og, P, xs, Qt in stress_run("fp32_ref", torch.float32, k):
         ref = O.newton_schulz(U, k)
-        ok = linear_gain(xs, k) * u <= 1e-2 if k > 5 else np.ones_like(xs, dtype=bool)
+        worst_whole = max(worst_whole, rel_fro(Og, ref))
+        ok = propagated_gain(xs, k) * u <= 1e-2 if k > 5 else np.ones_like(xs, dtype=bool)
         Pr, Qr = P[:, ok], Qt[ok, :].T
         err = rel_fro(Pr.T @ Og @ Qr, Pr.T @ ref @ Qr)
         D = Pr.T @ Og @ Qr
@@ -131,19 +167,20 @@ def test_stress_fp32_reference_mode(k):
         assert err < 1e-4, (s, err)
         assert diag_err < 1e-4 * max(1.0, np.linalg.norm(D)) and off < 1e-4, (s, diag_err, off)
         assert np.linalg.norm(Og, 2) <= PHI_MAX * (1 + 1e-4), s
+    print(f"stress fp32_ref k={k}: worst whole-matrix error against the oracle {worst_whole:.2e}")
 
 
 @pytest.mark.parametrize("k", [5, 10])
 def test_stress_bf16_singular_value_map(k):
     # bf16 operands round X, A and B to 8 bits: by Weyl's inequality each rounding of the
-    # normalised X moves every singular value by at most u = 2^-9, and k steps amplify an
-    # input perturbation of direction i by the gain of phi^k at s_i.  Directions with
+    # normalised X moves every singular value by at most u = 2^-9, and the later steps amplify
+    # that perturbation of direction i by their derivatives (propagated_gain).  Directions with
     # gain * u <= 1e-2 are resolvable; on them D = P^T O Q must follow the scalar
     # polynomial (3e-2) and O must match the oracle (2e-2).  Every direction, resolvable or
     # not, stays inside the quintic's invariant band [0, PHI_MAX] (to bf16 accuracy).
     u = 2.0 ** -9
     for s, U, Og, P, xs, Qt in stress_run("fast", torch.bfloat16, k):
-        ok = linear_gain(xs, k) * u <= 1e-2
+        ok = propagated_gain(xs, k) * u <= 1e-2
         Pr, Qr = P[:, ok], Qt[ok, :].T
         D = Pr.T @ Og @ Qr
         diag_err = np.max(np.abs(np.diag(D) - O.scalar_map(xs[ok], k))) if ok.any() else 0.0
@@ -152,7 +189,7 @@ def test_stress_bf16_singular_value_map(k):
         top = np.linalg.norm(Og, 2)
         print(f"stress bf16 {s} k={k}: {ok.sum()}/{len(xs)} resolvable, diag {diag_err:.2e}, "
               f"resolvable-subspace error {sub_err:.2e}, ||O||_2 {top:.4f}")
-        assert ok.sum() >= 16, (s, ok.sum())
+        assert ok.sum() >= 8, (s, ok.sum())
         assert diag_err < 3e-2, (s, diag_err)
         assert sub_err < 2e-2, (s, sub_err)
         assert top <= PHI_MAX * (1 + 4 * u), (s, top)
