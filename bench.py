@@ -44,7 +44,7 @@ def parse():
                          "split one set by matrix and all-gather the parameters (strong scaling)")
     ap.add_argument("--matrices", type=int, default=0,
                     help="use only the first N matrices of the workload (profiling captures of a smaller case)")
-    ap.add_argument("--schedule", choices=["auto", "staged", "fused"], default="auto",
+    ap.add_argument("--schedule", choices=["auto", "staged", "fused", "split"], default="auto",
                     help="Newton-Schulz launch schedule of the library (staged: one launch per stage)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -292,22 +292,24 @@ def kernel_table(prof, shapes, k, elem, steps, peaks, peak_src, wl_name):
     """
     fl = flops_by_kind(shapes, k)
     by = bytes_by_kind(shapes, elem)
-    kern = {kname: {"ms_total": ms, "launches": cnt, "ms_per_launch": (ms / cnt if cnt else None)}
+    kern = {kname: {"ms_total": ms, "launches": cnt, "ms_per_launch": (ms / cnt if cnt else None),
+                    "ms_per_step": ms / steps}
             for kname, (ms, cnt) in prof.items() if cnt}
-    per_launch_units = {
-        "gram": fl["gram"] / k if k else 0, "poly": fl["poly"] / k if k else 0,
-        "update": fl["update"] / k if k else 0,
+    # Algorithmic work of each kind per step; rates are work per step over that kind's time per
+    # step, so a kind that takes several launches per step (more than 192 matrices, more than six
+    # shape groups, the norm's finishing pass) is counted once.
+    per_step_units = {
+        "gram": fl["gram"], "poly": fl["poly"], "update": fl["update"],
         "momentum_norm": by["momentum_norm"], "write": by["write"],
-        "ns_small": sum(fl.values()),  # one launch runs every iteration of the step
-        "ns_fused": sum(fl.values()),
+        "ns_small": sum(fl.values()), "ns_fused": sum(fl.values()),
     }
     for kname, kd in kern.items():
         if kname in NS_KINDS:
-            kd["tflops"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e12
+            kd["tflops"] = per_step_units[kname] / (kd["ms_per_step"] * 1e-3) / 1e12
             kd["frac_of_burst_peak"] = kd["tflops"] / peaks["bf16_tflops"]
             kd["frac_of_sustained_peak"] = kd["tflops"] / peaks["bf16_tflops_sustained"]
         elif kname in ("momentum_norm", "write"):
-            kd["gbs"] = per_launch_units[kname] / (kd["ms_per_launch"] * 1e-3) / 1e9
+            kd["gbs"] = per_step_units[kname] / (kd["ms_per_step"] * 1e-3) / 1e9
             kd["frac_of_hbm"] = kd["gbs"] / peaks["hbm_gbs"]
     dominant = max(kern, key=lambda x: kern[x]["ms_total"])
     if dominant in NS_KINDS:

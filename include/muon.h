@@ -90,7 +90,8 @@ typedef struct {
   float lr;            /* learning rate */
   float beta;          /* momentum coefficient, 0 <= beta <= 1 */
   float weight_decay;  /* decoupled weight decay, applied to the pre-update W */
-  float eps;           /* added to ||X||_F before dividing, >= 0 */
+  float eps;           /* added to ||X||_F before dividing, >= 0; an all-zero X with
+                          eps = 0 is taken as the zero direction (zero update) */
   float a, b, c;       /* Newton-Schulz polynomial a x + b x^3 + c x^5 */
   int32_t nesterov;    /* nonzero: Nesterov blend */
   int32_t ns_steps;    /* iterations k, 0 <= k <= 64 */
@@ -208,6 +209,47 @@ MUON_API const char* muon_status_string(muon_status_t status);
 MUON_API muon_status_t muon_get_plan(muon_handle_t handle, int ns_steps, int* n_groups, int* launches_per_step);
 
 /*
+ * How the k Newton-Schulz iterations of a MUON_MODE_FAST handle are launched.
+ *   MUON_SCHEDULE_STAGED  one tensor-core launch per stage and iteration (3 k
+ *                         launches: Gram, polynomial, update), each over every
+ *                         matrix of the handle.
+ *   MUON_SCHEDULE_FUSED   all 3 k stages in one persistent launch: the tiles of
+ *                         every stage form one list, and a tile waits (on the
+ *                         device, bounded) only until the stage it reads is
+ *                         complete for its own matrix, so the stages of different
+ *                         matrices overlap and no launch boundary drains the GPU.
+ *                         Same arithmetic and rounding as STAGED (results are
+ *                         bitwise equal).  Needs at most 6 distinct shape groups.
+ *   MUON_SCHEDULE_SPLIT   the tiles of FUSED, one launch per stage (3 k launches):
+ *                         separates the single-launch kernel's tile machinery
+ *                         from its scheduling, for measurements.
+ *   MUON_SCHEDULE_AUTO    (default) the fastest for the handle's shapes.
+ * The small-matrix kernel (MUON_KERNEL_NS_SMALL) keeps precedence when its
+ * conditions hold; FP32_REF handles always run staged.  Returns
+ * MUON_ERR_UNSUPPORTED if FUSED is asked of a handle that cannot run it.
+ * The setting applies to later calls; it must not change while a captured graph
+ * of the handle is replayed.
+ */
+/*
+ * Host-only consistency check of the launch tables muon_step would build for
+ * these shapes on a device with num_sms SMs (no device needed): the persistent
+ * momentum/norm kernel's tile ranges and partial-sum slots, and the single-launch
+ * schedule's tile list for ns_steps iterations (every stage of every matrix
+ * covered once, stages listed before the tiles that wait for them, wait targets
+ * equal to the stages' tile counts), with and without the fused parameter
+ * write.  *problems receives the number of inconsistencies (0 when sound).  For
+ * tests and tools.
+ */
+MUON_API muon_status_t muon_check_plan(const muon_shape_t* shapes, int n, int ns_steps, int num_sms,
+                                       int64_t* problems);
+
+#define MUON_SCHEDULE_AUTO 0
+#define MUON_SCHEDULE_STAGED 1
+#define MUON_SCHEDULE_FUSED 2
+#define MUON_SCHEDULE_SPLIT 3
+MUON_API muon_status_t muon_set_schedule(muon_handle_t handle, int schedule);
+
+/*
  * Momentum, Nesterov blend and Frobenius norm of ONE matrix, with no workspace.
  * The pages have no counterpart for this entry point: it exists for callers that
  * cannot give this library device memory (a framework whose allocator must own
@@ -223,7 +265,9 @@ MUON_API muon_status_t muon_get_plan(muon_handle_t handle, int ns_steps, int* n_
  *   - rows * cols may be at most MUON_STATIC_MAX_ELEMENTS, else
  *     MUON_ERR_UNSUPPORTED is returned and nothing is enqueued.
  *   - The first call on a device (with that device current) looks up the
- *     array's device address; make it before capturing any stream.
+ *     array's device address; make it before capturing any stream.  A first
+ *     call on a stream that is being captured returns MUON_ERR_UNSUPPORTED
+ *     without touching the capture.
  *   - All calls share the array.  Calls in sequence on one stream are
  *     independent (the arrival counter is cleared at the start of each call);
  *     calls that overlap on the GPU race and give wrong norms.
@@ -265,7 +309,8 @@ MUON_API muon_status_t muon_get_group_buffers(muon_handle_t handle, int group, i
 #define MUON_KERNEL_WRITE 4
 #define MUON_KERNEL_SGEMM 5
 #define MUON_KERNEL_NS_SMALL 6 /* all iterations of a set of matrices of at most 256 x 256 */
-#define MUON_KERNEL_KINDS 7
+#define MUON_KERNEL_NS_FUSED 7 /* all iterations of a set in one launch (MUON_SCHEDULE_FUSED) */
+#define MUON_KERNEL_KINDS 8
 MUON_API muon_status_t muon_profile_begin(muon_handle_t handle, int max_steps);
 MUON_API muon_status_t muon_profile_end(muon_handle_t handle, double* ms, int* launches, int n_kinds);
 

@@ -28,7 +28,8 @@ STATUS = {
 MUON_OK, MUON_ERR_INVALID_ARG, MUON_ERR_UNSUPPORTED, MUON_ERR_CUDA = 0, 1, 2, 3
 MUON_ERR_WORKSPACE, MUON_ERR_TIMEOUT, MUON_ERR_DEVICE_STATUS, MUON_ERR_NO_DEVICE = 4, 5, 6, 7
 
-KERNEL_KINDS = ("momentum_norm", "gram", "poly", "update", "write", "sgemm_ref", "ns_small")
+KERNEL_KINDS = ("momentum_norm", "gram", "poly", "update", "write", "sgemm_ref", "ns_small", "ns_fused")
+MUON_SCHEDULE_AUTO, MUON_SCHEDULE_STAGED, MUON_SCHEDULE_FUSED, MUON_SCHEDULE_SPLIT = 0, 1, 2, 3
 
 
 class MuonError(RuntimeError):
@@ -100,6 +101,8 @@ def lib() -> ctypes.CDLL:
         L.muon_profile_end.argtypes = [_VP, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int),
                                        ctypes.c_int]
         L.muon_profile_end.restype = st
+        L.muon_set_schedule.argtypes = [_VP, ctypes.c_int]
+        L.muon_set_schedule.restype = st
         _lib = L
     return _lib
 
@@ -179,6 +182,21 @@ def muon_get_plan(handle: int, ns_steps: int):
     g, l = ctypes.c_int(0), ctypes.c_int(0)
     _check(lib().muon_get_plan(handle, ns_steps, ctypes.byref(g), ctypes.byref(l)), "muon_get_plan")
     return g.value, l.value
+
+
+def muon_check_plan(shapes, ns_steps: int, num_sms: int) -> int:
+    """Number of inconsistencies in the host-built launch tables (0 when sound); no device needed."""
+    L = lib()
+    f = L.muon_check_plan
+    f.argtypes = [ctypes.POINTER(Shape), ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
+    f.restype = ctypes.c_int
+    out = ctypes.c_int64(0)
+    _check(f(_shapes(shapes), len(shapes), int(ns_steps), int(num_sms), ctypes.byref(out)), "muon_check_plan")
+    return out.value
+
+
+def muon_set_schedule(handle: int, schedule: int) -> None:
+    _check(lib().muon_set_schedule(handle, int(schedule)), "muon_set_schedule")
 
 
 def muon_profile_begin(handle: int, max_steps: int) -> None:

@@ -7,13 +7,14 @@
 //    影响 paragraph).  It reads G and M once, writes M1 in place and U (cast to
 //    the Newton-Schulz operand type) into the zero-padded, oriented workspace
 //    buffer X0.  Tall matrices are transposed through shared memory so X0 is
-//    always min x max.  Each CTA handles two tiles.  The sum of squares is
-//    reduced warp -> CTA -> 8-CTA cluster (each CTA stores its partial into the
-//    rank-0 CTA's shared memory, one cluster barrier) -> one partial per
-//    cluster; the last cluster of a matrix to finish (acquire-release arrival
-//    counter) adds the partials in a fixed order, so the norm is
-//    deterministic, and stores ||U|| and 1/(||U|| + eps).  The normalisation itself is folded into the first
-//    Newton-Schulz products.
+//    always min x max.  The kernel is persistent (two CTAs per SM), CTA c
+//    taking every P-th tile from c on, with the next tile's loads in flight
+//    while it stores the current one.  The sum of squares goes warp -> one
+//    partial per (matrix, CTA, warp) in the workspace; norm_finish_kernel, the
+//    next launch, adds each matrix's partials in a fixed order, so the norm is
+//    deterministic, and stores ||U|| and 1/(||U|| + eps) (0 when both are 0: a
+//    zero direction gives a zero update).  The normalisation itself is folded
+//    into the first Newton-Schulz products.
 //
 //  * param_write_kernel — the parameter write
 //    W1 = (1 - lr*wd) W - lr*sqrt(max(1, rows/cols)) O, O the final X oriented
@@ -24,6 +25,9 @@
 // accesses whenever a row segment is aligned and complete, and element-wise
 // accesses on ragged edges.
 #include <cuda_bf16.h>
+
+#include <algorithm>
+#include <vector>
 
 #include "muon_device.cuh"
 #include "muon_internal.h"
@@ -85,15 +89,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
-}
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 template <typename Mats>
@@ -210,22 +205,32 @@ __device__ __forceinline__ void momentum_chunk(const EwMat& mt, const EwParams& 
   for (int i = 0; i < 8; ++i) ss = fmaf(u[i], u[i], ss);
 }
 
-// One 64 x 128 tile of the oriented X0: momentum/Nesterov on the matching source
-// elements, U stored to X0 (transposed through shared memory for tall matrices);
-// returns this thread's sum of squares.
+// The loads of one 64 x 128 tile of the oriented X0 (the matching source elements of G and M,
+// whole aligned 8-element vectors only; ragged edges are read by momentum_chunk itself).
+template <typename T>
+__device__ __forceinline__ void momentum_tile_load(const EwMat& mt, const EwParams& p, int t, MomentumChunks<T>& ch) {
+  const int xr0 = (t / mt.tiles_c) * kEwTileR;
+  const int xc0 = (t % mt.tiles_c) * kEwTileC;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = threadIdx.x + q * kEwThreads;
+    if (!mt.trans)
+      momentum_load<T>(mt, p, q, xr0 + (c >> 4), xc0 + (c & 15) * 8, ch);
+    else  // source tile in the caller's layout: rows xc0.., cols xr0..
+      momentum_load<T>(mt, p, q, xc0 + (c >> 3), xr0 + (c & 7) * 8, ch);
+  }
+}
+
+// The rest of the tile once its loads are in `ch`: momentum/Nesterov, M1 stored, U stored to X0
+// (transposed through shared memory for tall matrices); returns this thread's sum of squares.
 template <typename T, typename XT, int LD>
-__device__ __forceinline__ float momentum_tile(const EwMat& mt, const EwParams& p, int t, XT (*stage)[LD]) {
+__device__ __forceinline__ float momentum_tile_store(const EwMat& mt, const EwParams& p, int t,
+                                                     const MomentumChunks<T>& ch, XT (*stage)[LD]) {
   float ss = 0.0f;
   const int xr0 = (t / mt.tiles_c) * kEwTileR;
   const int xc0 = (t % mt.tiles_c) * kEwTileC;
   XT* x = static_cast<XT*>(mt.x);
-  MomentumChunks<T> ch;
   if (!mt.trans) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = threadIdx.x + q * kEwThreads;
-      momentum_load<T>(mt, p, q, xr0 + (c >> 4), xc0 + (c & 15) * 8, ch);
-    }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int c = threadIdx.x + q * kEwThreads;
@@ -235,12 +240,6 @@ __device__ __forceinline__ float momentum_tile(const EwMat& mt, const EwParams& 
       Vec8<XT>::store(x + static_cast<size_t>(xr0 + r) * mt.np + xc0 + cc, u);
     }
   } else {
-    // source tile in the caller's layout: rows xc0.., cols xr0..
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = threadIdx.x + q * kEwThreads;
-      momentum_load<T>(mt, p, q, xc0 + (c >> 3), xr0 + (c & 7) * 8, ch);
-    }
     __syncthreads();  // the previous tile's staged values have been read out
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -265,68 +264,103 @@ __device__ __forceinline__ float momentum_tile(const EwMat& mt, const EwParams& 
   return ss;
 }
 
+// The matrix of tile t, starting the search at matrix mi (t never lies before it).
+__device__ __forceinline__ int matrix_of_tile(const EwParams& p, int mi, int t) {
+  while (mi + 1 < p.nmat && t >= p.mat[mi + 1].tile_begin) ++mi;
+  return mi;
+}
+
+// This warp's part of matrix mt's sum of squares (the tiles this CTA took from mt) is complete:
+// one plain store into the warp's own slot.  CTA c reaches the tiles of mt whose index is
+// congruent to c modulo the grid, the first at offset r = (c - tile_begin) mod grid < nparts,
+// so slot (r, warp) is written by this warp alone.  No atomics and no fences: the sums are added
+// by norm_finish_kernel, the next launch on the stream.
+__device__ __forceinline__ void momentum_flush(const EwParams& p, const EwMat& mt, float ss) {
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) {
+    const int g = static_cast<int>(gridDim.x);
+    const int r = ((static_cast<int>(blockIdx.x) - mt.tile_begin) % g + g) % g;
+    p.partials[static_cast<size_t>(mt.part_begin + r) * (kEwThreads / 32) + (threadIdx.x >> 5)] = ss;
+  }
+}
+
+// Persistent: CTA c takes tiles c, c + P, c + 2P, ... of the launch (T tiles, P CTAs, matrices
+// back to back), so at any moment the CTAs work on neighbouring tiles (the same rows of the same
+// matrix, which keeps the DRAM pages they touch open) rather than on P distant streams.  For bf16
+// sources the loads of the next tile are issued before the current tile is computed and stored
+// (two register buffers), so every thread keeps eight 16-byte loads in flight while it works.
 template <typename T, typename XT>
-__global__ void __cluster_dims__(kEwCluster, 1, 1) __launch_bounds__(kEwThreads, 3)
-    momentum_norm_kernel(const __grid_constant__ EwParams p) {
+__global__ void __launch_bounds__(kEwThreads, kEwCtasPerSm) momentum_norm_kernel(const __grid_constant__ EwParams p) {
   constexpr int LD = kEwTileC + (sizeof(XT) == 2 ? 2 : 1);
   __shared__ XT stage[kEwTileR][LD];
-  __shared__ float red[kEwThreads / 32];
-  __shared__ float slots[kEwCluster];  // used in the cluster's rank-0 CTA: one partial per CTA
 
-  const int cta = blockIdx.x;
-  const EwMat& mt = p.mat[find_matrix(p.mat, p.nmat, cta)];
-  const int local = cta - mt.tile_begin;  // CTA index within the matrix
+  const int step = static_cast<int>(gridDim.x);
+  const int t0 = static_cast<int>(blockIdx.x);
+  if (t0 >= p.total_tiles) return;
+  int lo = 0, hi = p.nmat - 1;  // matrix of t0
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.mat[mid].tile_begin <= t0) lo = mid; else hi = mid - 1;
+  }
+  int mi = lo;          // matrix whose partial sum is being accumulated
   float ss = 0.0f;
+  // bf16 sources: two register buffers (the next tile's loads in flight); fp32 sources hold
+  // twice the bytes per tile, so they keep one buffer and rely on the second resident CTA.
+  constexpr int NBUF = sizeof(T) == 2 ? 2 : 1;
+  MomentumChunks<T> buf[NBUF];
+  int mnext = mi;
+  if (NBUF == 2) momentum_tile_load<T>(p.mat[mi], p, t0 - p.mat[mi].tile_begin, buf[0]);
 #pragma unroll 1
-  for (int j = 0; j < kEwTilesPerCta; ++j) {
-    const int t = local * kEwTilesPerCta + j;
-    if (t < mt.ntiles) ss += momentum_tile<T, XT, LD>(mt, p, t, stage);
-  }
-
-  // CTA reduction (fixed order)
-  ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  const uint32_t rank = cluster_ctarank();
-  if (threadIdx.x == 0) {
-    float s = 0.0f;
+  for (int t = t0; t < p.total_tiles; t += NBUF * step) {
 #pragma unroll
-    for (int w = 0; w < kEwThreads / 32; ++w) s += red[w];
-    // push this CTA's partial into its slot in the rank-0 CTA's shared memory
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(remote) : "r"(smem_u32(&slots[rank])));
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(s) : "memory");
-  }
-  // One cluster barrier: every partial has landed in rank 0 before it reads them, and no
-  // CTA touches another CTA's shared memory afterwards.
-  cluster_sync_all();
-  if (rank == 0 && threadIdx.x < 32) {
-    unsigned int prev = 0;
-    if (threadIdx.x == 0) {
-      float s = 0.0f;
-#pragma unroll
-      for (int r = 0; r < kEwCluster; ++r) s += slots[r];
-      p.partials[mt.part_begin + local / kEwCluster] = s;
-      // release the partial, acquire the others' if this cluster is the matrix's last
-      asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                   : "=r"(prev)
-                   : "l"(p.counters + mt.scal_idx)
-                   : "memory");
-    }
-    __syncwarp();
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    if (prev == static_cast<unsigned int>(mt.nclusters - 1)) {
-      float s = 0.0f;
-      for (int i = threadIdx.x; i < mt.nclusters; i += 32) s += __ldcg(&p.partials[mt.part_begin + i]);
-      s = warp_sum(s);
-      if (threadIdx.x == 0) {
-        const float nrm = sqrtf(s);
-        p.scal[2 * mt.scal_idx] = nrm;
-        p.scal[2 * mt.scal_idx + 1] = 1.0f / (nrm + p.eps);
-        p.norms[mt.caller_idx] = nrm;
-        p.counters[mt.scal_idx] = 0u;
+    for (int h = 0; h < NBUF; ++h) {
+      const int tt = t + h * step;
+      if (tt < p.total_tiles) {
+        int mcur;
+        if (NBUF == 2) {
+          mcur = mnext;
+          if (tt + step < p.total_tiles) {
+            mnext = matrix_of_tile(p, mcur, tt + step);
+            momentum_tile_load<T>(p.mat[mnext], p, tt + step - p.mat[mnext].tile_begin, buf[(h + 1) % NBUF]);
+          }
+        } else {
+          mcur = matrix_of_tile(p, mi, tt);
+          momentum_tile_load<T>(p.mat[mcur], p, tt - p.mat[mcur].tile_begin, buf[0]);
+        }
+        if (mcur != mi) {
+          momentum_flush(p, p.mat[mi], ss);
+          ss = 0.0f;
+          mi = mcur;
+        }
+        ss += momentum_tile_store<T, XT, LD>(p.mat[mi], p, tt - p.mat[mi].tile_begin, buf[h], stage);
       }
     }
+  }
+  momentum_flush(p, p.mat[mi], ss);
+}
+
+// The norms of one momentum/norm launch's matrices: CTA j adds matrix j's per-warp partial sums
+// in a fixed order (so the norm is the same on every run), and stores ||U|| and 1/(||U|| + eps)
+// (0 when both are 0: a zero direction gives a zero update).
+__global__ void __launch_bounds__(kEwThreads) norm_finish_kernel(const __grid_constant__ EwParams p) {
+  __shared__ float red[kEwThreads / 32];
+  const EwMat& mt = p.mat[blockIdx.x];
+  const int n = mt.nparts * (kEwThreads / 32);
+  const float* src = p.partials + static_cast<size_t>(mt.part_begin) * (kEwThreads / 32);
+  float s = 0.0f;
+  for (int i = threadIdx.x; i < n; i += kEwThreads) s += src[i];
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kEwThreads / 32; ++w) t += red[w];
+    const float nrm = sqrtf(t);
+    const float den = nrm + p.eps;
+    p.scal[2 * mt.scal_idx] = nrm;
+    p.scal[2 * mt.scal_idx + 1] = den > 0.0f ? 1.0f / den : 0.0f;
+    p.norms[mt.caller_idx] = nrm;
   }
 }
 
@@ -431,7 +465,10 @@ __global__ void __launch_bounds__(kEwThreads, 3) param_write_kernel(const __grid
 
 template <typename T, typename XT>
 cudaError_t launch_mn(const EwParams& p, cudaStream_t s) {
-  momentum_norm_kernel<T, XT><<<p.total_ctas, kEwThreads, 0, s>>>(p);
+  momentum_norm_kernel<T, XT><<<p.grid, kEwThreads, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  norm_finish_kernel<<<p.nmat, kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 template <typename T, typename XT>
@@ -442,8 +479,45 @@ cudaError_t launch_wr(const WrParams& p, cudaStream_t s) {
 
 }  // namespace
 
+long long check_front_tables(const EwParams& p) {
+  // Replay the persistent kernel's walk on the host: the matrices' tile ranges back to back, and
+  // each matrix's partial sums written once per CTA that reaches it (the CTA's first tile of the
+  // matrix at offset r < nparts) into slots [part_begin, part_begin + nparts), no slot twice.
+  long long bad = 0;
+  if (p.nmat < 1 || p.nmat > kEwMatsPerLaunch || p.grid < 1 || p.grid > kEwMaxCtas || p.grid > p.total_tiles)
+    return 1;
+  int tiles = 0, parts = 0;
+  for (int j = 0; j < p.nmat; ++j) {
+    const EwMat& m = p.mat[j];
+    if (m.tile_begin != tiles || m.ntiles < 1 || m.part_begin != parts || m.nparts != std::min(m.ntiles, p.grid) ||
+        m.tiles_c * kEwTileC != m.np || m.ntiles * kEwTileR * kEwTileC != m.mp * m.np)
+      ++bad;
+    tiles += m.ntiles;
+    parts += m.nparts;
+  }
+  if (tiles != p.total_tiles) ++bad;
+  std::vector<int> written(static_cast<size_t>(parts > 0 ? parts : 1), 0);
+  for (int c = 0; c < p.grid; ++c) {
+    int mi = -1;
+    for (int t = c; t < p.total_tiles; t += p.grid) {
+      int mt = 0;
+      while (mt + 1 < p.nmat && t >= p.mat[mt + 1].tile_begin) ++mt;
+      if (mt != mi) {  // this CTA's flush of matrix mt
+        const EwMat& m = p.mat[mt];
+        const int r = ((c - m.tile_begin) % p.grid + p.grid) % p.grid;
+        if (r != t - m.tile_begin || r >= m.nparts) ++bad;
+        else ++written[m.part_begin + r];
+        mi = mt;
+      }
+    }
+  }
+  for (int i = 0; i < parts; ++i)
+    if (written[i] != 1) ++bad;
+  return bad;
+}
+
 cudaError_t launch_momentum_norm(const EwParams& p, Dtype io, Dtype xt, cudaStream_t s) {
-  if (p.total_ctas <= 0) return cudaSuccess;
+  if (p.total_tiles <= 0 || p.grid <= 0) return cudaSuccess;
   if (io == kBF16 && xt == kBF16) return launch_mn<__nv_bfloat16, __nv_bfloat16>(p, s);
   if (io == kF32 && xt == kBF16) return launch_mn<float, __nv_bfloat16>(p, s);
   if (io == kBF16 && xt == kF32) return launch_mn<__nv_bfloat16, float>(p, s);

@@ -12,7 +12,8 @@
 //
 // Set-up: the first call on a device (with that device current) looks up the
 // array's device address with cudaGetSymbolAddress and caches it; make that
-// first call before capturing any stream.  Every call shares the one array and
+// first call before capturing any stream.  A first call made on a stream that
+// is being captured returns MUON_ERR_UNSUPPORTED and leaves the capture intact.  Every call shares the one array and
 // leaves its last contents behind; the counter is cleared at the start of each
 // call, so calls in sequence are independent, but calls that overlap on the GPU
 // (different streams, or graphs replayed concurrently) race on the array.
@@ -154,20 +155,23 @@ constexpr int kMaxDevices = 64;
 unsigned char* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-cudaError_t scratch_for_current_device(unsigned char** out) {
+// Returns MUON_OK, MUON_ERR_UNSUPPORTED when the address is not known yet and `stream` is being
+// captured (the look-up would break the capture), or MUON_ERR_CUDA.
+muon_status_t scratch_for_current_device(cudaStream_t stream, unsigned char** out) {
   int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MUON_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (g_scratch_addr[dev] == nullptr) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return MUON_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return MUON_ERR_UNSUPPORTED;
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_norm_scratch);
-    if (e != cudaSuccess) return e;
+    if (cudaGetSymbolAddress(&p, g_norm_scratch) != cudaSuccess) return MUON_ERR_CUDA;
     g_scratch_addr[dev] = static_cast<unsigned char*>(p);
   }
   *out = g_scratch_addr[dev];
-  return cudaSuccess;
+  return MUON_OK;
 }
 
 }  // namespace
@@ -183,9 +187,10 @@ extern "C" MUON_API muon_status_t muon_momentum_norm_static(const void* G, void*
   if (rows > MUON_STATIC_MAX_ELEMENTS / cols) return MUON_ERR_UNSUPPORTED;  // beyond the fixed scratch
   const long long n = rows * cols;
   unsigned char* scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != cudaSuccess) {
+  const muon_status_t st = scratch_for_current_device(stream, &scratch);
+  if (st != MUON_OK) {
     cudaGetLastError();
-    return MUON_ERR_CUDA;
+    return st;
   }
   const long long ctas = (n + kPerCta - 1) / kPerCta;
   const int grid = static_cast<int>((ctas + kCluster - 1) / kCluster * kCluster);

@@ -73,21 +73,24 @@ constexpr uint32_t A_STAGE = BM * BK * 2;               // 16 KB: this CTA's 128
 constexpr uint32_t B_STAGE = (BN / 2) * BK * 2;         // 16 KB: this CTA's half of B
 constexpr uint32_t TMEM_COLS = 512;                     // 2 accumulators x 256 fp32 columns
 constexpr uint32_t BAR_BYTES = 256;
-constexpr int EPI_PITCH = 40;                            // staged aux row: 32 bf16 + 8 pad (80 B, 16-B aligned)
 constexpr int F32_PITCH = 36;                            // staged fp32 row: 32 + 4 pad (144 B, 16-B aligned)
 constexpr int EPI_WARPS = kTcEpiWarps;
 // Shared memory: the stage ring (at most 144 KB: 4 x 32 KB for 256-wide tiles, 3 x 48 KB
 // for 512-wide ones), then per epilogue warp two 32 x 32 bf16 store tiles (2 KB each,
-// 64-byte swizzle), then per warp the auxiliary chunk.  The fp32 staging of the fused
-// parameter write reuses the start of the region (that launch makes no TMA stores).
+// 64-byte swizzle), then per warp two 32 x 32 chunks of the polynomial's input A, loaded by
+// TMA two chunks ahead (same 64-byte swizzle).  The fp32 staging of the fused parameter write
+// reuses the start of the region (that launch makes no TMA stores and reads no A).
 constexpr uint32_t STAGE_REGION = 147456;
 constexpr uint32_t EPI_OUT_BYTES = 2048;
-constexpr uint32_t EPI_AUX_BYTES = 32 * EPI_PITCH * 2;
+constexpr uint32_t EPI_AUX_BYTES = 2048;
 constexpr uint32_t EPI_F32_BYTES = 32 * F32_PITCH * 4;
 constexpr uint32_t EPI_OFFSET = STAGE_REGION;            // 1024-byte aligned, as the swizzled tiles need
 constexpr uint32_t EPI_AUX_OFFSET = EPI_OFFSET + EPI_WARPS * 2 * EPI_OUT_BYTES;
-constexpr uint32_t BAR_OFFSET = EPI_AUX_OFFSET + EPI_WARPS * EPI_AUX_BYTES;
+constexpr uint32_t BAR_OFFSET = EPI_AUX_OFFSET + EPI_WARPS * 2 * EPI_AUX_BYTES;
 constexpr size_t SMEM_BYTES = 1024 + BAR_OFFSET + BAR_BYTES;
+// barriers: full[NST], empty[NST], accf[2], acce[2], the TMEM slot word, then two per epilogue
+// warp for its A chunks
+static_assert((2 * kTcStages + 5 + 2 * kTcEpiWarps) * 8 <= BAR_BYTES, "barriers must fit their region");
 static_assert(EPI_WARPS * EPI_F32_BYTES <= BAR_OFFSET - EPI_OFFSET, "fp32 staging must fit the epilogue region");
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
@@ -164,6 +167,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * NST + 2 + a); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NST + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto aux_bar = [&](int w, int j) { return bar0 + 8u * (2 * NST + 5 + 2 * w + j); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();           // 0: issues the MMAs; 1: its peer
@@ -179,6 +183,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       mbar_init(accf_bar(a), 1);   // one multicast commit
       mbar_init(acce_bar(a), 2 * EPI_WARPS);   // one arrival per epilogue warp of both CTAs
     }
+    for (int w = 0; w < EPI_WARPS; ++w)
+      for (int j = 0; j < 2; ++j) mbar_init(aux_bar(w, j), 1);  // the warp's arrive.expect_tx
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -188,6 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       tma_prefetch_desc(&p.g[g].tm_at);
       tma_prefetch_desc(&p.g[g].tm_b);
       tma_prefetch_desc(&p.g[g].tm_bt);
+      if (KIND == kPoly) tma_prefetch_desc(&p.g[g].tm_aux);
     }
   }
   if (warp == 1) {
@@ -331,18 +338,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     const int ch0 = (e >> 2) * NW;          // this warp's first chunk
     uint8_t* otile = smem + EPI_OFFSET + e * 2 * EPI_OUT_BYTES;
     const uint32_t otile_u32 = smem_u32(otile);
-    __nv_bfloat16* stg_aux = reinterpret_cast<__nv_bfloat16*>(smem + EPI_AUX_OFFSET + e * EPI_AUX_BYTES);
+    const uint8_t* abuf = smem + EPI_AUX_OFFSET + e * 2 * EPI_AUX_BYTES;  // this warp's two A chunks
+    const uint32_t abuf_u32 = smem_u32(abuf);
     float* st32 = reinterpret_cast<float*>(smem + EPI_OFFSET + e * EPI_F32_BYTES);
     const int sub_r = lane >> 2, sub_c = (lane & 3) * 8;
     const int swz = (lane >> 1) & 3;  // 64-byte swizzle of this lane's staging row
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = cl; t < p.total_tiles; t += ncl) {
+    uint32_t naux = 0;                // A chunks this warp has consumed (their buffers alternate)
+    uint32_t nissued = 0;             // A chunks lane 0 has requested
+    bool aux_ok = true;
+    for (int t = cl; t < p.total_tiles && aux_ok; t += ncl) {
       const Tile ti = decode_tile<KIND, TW>(p, t);
       const TcGroup& G = p.g[ti.g];
-      const int ld = G.out_ld;
-      const size_t mat_off = static_cast<size_t>(ti.mat) * G.mp * ld;
-      const __nv_bfloat16* aux = G.aux ? static_cast<const __nv_bfloat16*>(G.aux) + mat_off : nullptr;
+      const bool aux = KIND == kPoly;   // the polynomial's b A + a I reads A
       const int gr0 = ti.row0 + static_cast<int>(rank) * BM + quad * 32;  // first row of this warp
       const int gr = gr0 + lane;
       // Fused parameter write (last Update): the caller's matrix of this tile.
@@ -363,22 +372,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       auto woff = [&](int gc, int rr) -> size_t {
         return tr ? static_cast<size_t>(gc + rr) * ldw + gr0 + sub_c : static_cast<size_t>(gr0 + rr) * ldw + gc + sub_c;
       };
-      // The auxiliary input (A for Poly, W for the fused Update) does not depend on the
-      // accumulator: fetch the warp's first chunk before waiting, and every later chunk
-      // one step ahead, so its latency hides behind the accumulator drain.
+      // The auxiliary inputs do not depend on the accumulator, so they are fetched before
+      // waiting for it: the polynomial's chunks of A by TMA into the warp's two A buffers (the
+      // first two now, each later one as soon as the buffer two chunks back is read), the W of
+      // the fused parameter write into registers one chunk ahead.
+      auto aux_issue = [&](int c) {  // lane 0: chunk c of this warp into buffer (naux + c) & 1
+        const uint32_t n = naux + static_cast<uint32_t>(c);
+        ++nissued;
+        mbar_arrive_expect_tx(aux_bar(e, n & 1), EPI_AUX_BYTES);
+        tma_load_3d(abuf_u32 + (n & 1) * EPI_AUX_BYTES, &G.tm_aux, aux_bar(e, n & 1), ti.col0 + (ch0 + c) * 32, gr0,
+                    ti.mat);
+      };
+      if (aux && lane == 0) {
+        aux_issue(0);
+        if (NW > 1) aux_issue(1);
+      }
       uint4 pf[4];
       auto pre_load = [&](int ch, uint4 (&dst)[4]) {
         const int gc = ti.col0 + ch * 32;
-        if (aux != nullptr) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = __ldg(reinterpret_cast<const uint4*>(aux + static_cast<size_t>(gr0 + q * 8 + sub_r) * ld + gc + sub_c));
-        } else if (wread && gc < G.n_real) {
+        if (wread && gc < G.n_real) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) dst[q] = __ldcs(reinterpret_cast<const uint4*>(W + woff(gc, q * 8 + sub_r)));
         }
       };
-      const bool has_pre = aux != nullptr || wread;
+      const bool has_pre = wread;
       if (has_pre) pre_load(ch0, pf);
       if (!mbar_wait_bounded(accf_bar(acc), acc_phase, tmo, abort_flag, p.status)) break;
       tc_fence_after();
@@ -442,18 +459,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           for (int q = 0; q < 4; ++q) pf[q] = nx[q];
           continue;
         }
-        if (aux != nullptr) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(stg_aux + (q * 8 + sub_r) * EPI_PITCH + sub_c) = pf[q];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) pf[q] = nx[q];
-          __syncwarp();
+        if (aux) {
+          // this lane's row of the chunk of A (64-byte rows, 64-byte swizzle, as TMA wrote them)
+          const uint32_t n = naux + static_cast<uint32_t>(c);
+          if (!mbar_wait_bounded(aux_bar(e, n & 1), (n >> 1) & 1u, tmo, abort_flag, p.status)) {
+            aux_ok = false;
+            break;
+          }
+          const uint8_t* arow = abuf + (n & 1) * EPI_AUX_BYTES + lane * 64;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float a8[8];
-            unpack8(*reinterpret_cast<const uint4*>(stg_aux + lane * EPI_PITCH + q * 8), a8);
+            unpack8(*reinterpret_cast<const uint4*>(arow + ((q ^ swz) << 4)), a8);
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[8 * q + i] = s * fmaf(p.c_acc, v[8 * q + i], p.c_aux * a8[i]);
+          }
+          // every lane has used its row: the buffer may take the chunk two ahead
+          __syncwarp();
+          if (lane == 0 && c + 2 < NW) {
+            fence_async_smem();
+            aux_issue(c + 2);
           }
         } else {
 #pragma unroll
@@ -479,6 +504,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           bulk_commit();
         }
       }
+      if (aux) naux += NW;  // (an early exit leaves naux behind nissued; see the drain below)
       if (++acc == NACC) {
         acc = 0;
         acc_phase ^= 1u;
@@ -486,6 +512,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     }
     // every TMA store of this warp has finished (its shared memory read, its global write)
     if (lane == 0) bulk_wait_all();
+    // after an early exit, A chunks may still be on their way into this warp's buffers: wait
+    // (bounded) for them before the CTA leaves
+    if (KIND == kPoly && lane == 0) {
+      for (uint32_t n = naux; n < nissued; ++n)
+        (void)mbar_wait_bounded(aux_bar(e, n & 1), (n >> 1) & 1u, tmo, nullptr, p.status);
+    }
     __syncwarp();
   }
 

@@ -60,10 +60,9 @@ struct GroupPlan {
 struct Plan {
   std::vector<GroupPlan> groups;
   std::vector<int> mat_group, mat_slot, scal_idx;
-  std::vector<int> ew_ntiles, ew_nclusters, ew_part_begin;
-  size_t off_status, off_counters, off_scal, off_norms, off_partials;
+  std::vector<int> ew_ntiles;
+  size_t off_status, off_deps, off_scal, off_norms, off_partials;
   size_t total;
-  int total_parts;
 };
 
 bool shapes_ok(const muon_shape_t* shapes, int n) {
@@ -121,24 +120,20 @@ void make_plan(const muon_shape_t* shapes, int n, muon_mode_t mode, Plan* P) {
     base += gp.cnt;
   }
   P->ew_ntiles.assign(n, 0);
-  P->ew_nclusters.assign(n, 0);
-  P->ew_part_begin.assign(n, 0);
-  int parts = 0;
   for (int i = 0; i < n; ++i) {
     const GroupPlan& gp = P->groups[P->mat_group[i]];
-    const int nt = (gp.mp / kEwTileR) * (gp.np / kEwTileC);
-    P->ew_ntiles[i] = nt;
-    constexpr int per_cluster = kEwCluster * kEwTilesPerCta;
-    P->ew_nclusters[i] = (nt + per_cluster - 1) / per_cluster;
-    P->ew_part_begin[i] = parts;
-    parts += P->ew_nclusters[i];
+    P->ew_ntiles[i] = (gp.mp / kEwTileR) * (gp.np / kEwTileC);
   }
-  P->total_parts = parts;
+  // One partial sum per (matrix, CTA, warp) of the persistent momentum/norm kernel, min(ntiles,
+  // grid) CTAs per matrix; launches in sequence reuse the buffer, so the whole set bounds it.
+  size_t parts = 0;
+  for (int i = 0; i < n; ++i) parts += static_cast<size_t>(std::min(P->ew_ntiles[i], kEwMaxCtas)) * (kEwThreads / 32);
   size_t off = 0;
   P->off_status = off;
   off = align_up(off + 64, 1024);
-  P->off_counters = off;
-  off = align_up(off + sizeof(unsigned int) * n, 1024);
+  // the single-launch schedule's completion counters, [3 k][n] for k up to 64
+  P->off_deps = off;
+  off = align_up(P->off_deps + sizeof(unsigned int) * 3 * 64 * static_cast<size_t>(n), 1024);
   P->off_scal = off;
   off = align_up(off + sizeof(float) * 2 * n, 1024);
   P->off_norms = off;
@@ -257,16 +252,17 @@ struct muon_ctx {
   char* ws = nullptr;
   size_t ws_bytes = 0;
   unsigned int* d_status = nullptr;
-  unsigned int* d_counters = nullptr;
   float* d_scal = nullptr;
   float* d_partials = nullptr;
   float* d_norms = nullptr;   // ||U_i||_F in caller order
   bool fuse_shapes_ok = false;  // every group's real dimensions are multiples of 32, n <= kTcMaxFused
+  int schedule = MUON_SCHEDULE_AUTO;
   // launch parameter blocks (tens of KB), reused by every call on this handle
   EwParams ew;
   WrParams wr;
   TcParams tc;
   SmallParams sm;
+  NsParams ns;
   // tracing (muon_profile_begin / muon_profile_end)
   int prof_steps_left = 0;
   std::vector<std::pair<int, cudaEvent_t>> prof_events;  // kind (-1: start of a call), event
@@ -292,6 +288,55 @@ void trace_call_end(muon_ctx* h) {
   if (h->prof_steps_left > 0) --h->prof_steps_left;
 }
 
+bool small_path(const muon_ctx* h, int k);
+
+// Whether the k iterations run as one launch (all stages, per-matrix completion counters)
+// rather than one launch per stage: FAST mode, at most kTcMaxGroups shape groups, not the
+// small-matrix kernel's sets, and the handle's schedule allows it.
+bool fused_possible(const muon_ctx* h, int k) {
+  return h->mode == MUON_MODE_FAST && k >= 1 && !h->plan.groups.empty() &&
+         h->plan.groups.size() <= static_cast<size_t>(kTcMaxGroups) && !small_path(h, k);
+}
+bool fused_schedule(const muon_ctx* h, int k) {
+  if (!fused_possible(h, k)) return false;
+  return h->schedule == MUON_SCHEDULE_FUSED || h->schedule == MUON_SCHEDULE_SPLIT;
+}
+
+// Tile tables of one momentum/norm launch (matrices b .. b+cnt-1), without the pointers and the
+// hyper-parameters: the persistent grid of num_sms * kEwCtasPerSm CTAs, CTA c taking tiles
+// c, c + G, ... of the launch's T tiles; a matrix gets one partial sum per warp of every CTA
+// that reaches it, min(ntiles, G) CTAs.
+void front_tables(const Plan& P, const std::vector<muon_shape_t>& shapes, int b, int cnt, int num_sms,
+                  EwParams* prm) {
+  std::memset(prm, 0, sizeof(*prm));
+  prm->nmat = cnt;
+  int total = 0;
+  for (int j = 0; j < cnt; ++j) total += P.ew_ntiles[b + j];
+  const int grid = std::max(1, std::min({num_sms * kEwCtasPerSm, kEwMaxCtas, total}));
+  prm->total_tiles = total;
+  prm->grid = grid;
+  int tiles = 0, parts = 0;
+  for (int j = 0; j < cnt; ++j) {
+    const int i = b + j;
+    const GroupPlan& gp = P.groups[P.mat_group[i]];
+    EwMat& m = prm->mat[j];
+    m.rows = static_cast<int>(shapes[i].rows);
+    m.cols = static_cast<int>(shapes[i].cols);
+    m.mp = gp.mp;
+    m.np = gp.np;
+    m.trans = shapes[i].rows > shapes[i].cols ? 1 : 0;
+    m.tile_begin = tiles;
+    m.tiles_c = gp.np / kEwTileC;
+    m.ntiles = P.ew_ntiles[i];
+    m.scal_idx = P.scal_idx[i];
+    m.caller_idx = i;
+    m.nparts = std::min(m.ntiles, grid);
+    m.part_begin = parts;
+    parts += m.nparts;
+    tiles += m.ntiles;
+  }
+}
+
 // The elementwise front end (momentum + norm + orientation) over all matrices.
 cudaError_t enqueue_front(muon_ctx* h, const void* const* src, void* const* mom, const muon_hparams_t* hp,
                           cudaStream_t st, int* launches) {
@@ -299,22 +344,24 @@ cudaError_t enqueue_front(muon_ctx* h, const void* const* src, void* const* mom,
   const Plan& P = h->plan;
   const Dtype io = (h->dtype == MUON_BF16) ? kBF16 : kF32;
   const Dtype xt = (h->mode == MUON_MODE_FAST) ? kBF16 : kF32;
-  cudaError_t e = cudaMemsetAsync(h->d_counters, 0, sizeof(unsigned int) * h->n, st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (fused_schedule(h, hp->ns_steps)) {
+    // the single-launch schedule's stage completion counters start at zero
+    e = cudaMemsetAsync(h->ws + P.off_deps, 0, sizeof(unsigned int) * 3 * hp->ns_steps * static_cast<size_t>(h->n), st);
+    if (e != cudaSuccess) return e;
+  }
   trace(h, -1, st);  // start of the traced kernel sequence of this call
   EwParams& prm = h->ew;
   for (int b = 0; b < h->n; b += kEwMatsPerLaunch) {
     const int cnt = std::min(kEwMatsPerLaunch, h->n - b);
-    std::memset(&prm, 0, sizeof(prm));
-    prm.nmat = cnt;
+    front_tables(P, h->shapes, b, cnt, h->num_sms, &prm);
     prm.beta = hp->beta;
     prm.eps = hp->eps;
     prm.nesterov = hp->nesterov ? 1 : 0;
     prm.partials = h->d_partials;
     prm.scal = h->d_scal;
-    prm.counters = h->d_counters;
     prm.norms = h->d_norms;
-    int vec_ok = 1, tiles = 0;
+    int vec_ok = 1;
     for (int j = 0; j < cnt; ++j) {
       const int i = b + j;
       const GroupPlan& gp = P.groups[P.mat_group[i]];
@@ -323,30 +370,62 @@ cudaError_t enqueue_front(muon_ctx* h, const void* const* src, void* const* mom,
       m.src = src[i];
       m.mom = mom ? mom[i] : nullptr;
       m.x = h->ws + gp.off_x[0] + static_cast<size_t>(P.mat_slot[i]) * gp.mp * gp.np * elem;
-      m.rows = static_cast<int>(h->shapes[i].rows);
-      m.cols = static_cast<int>(h->shapes[i].cols);
-      m.mp = gp.mp;
-      m.np = gp.np;
-      m.trans = h->shapes[i].rows > h->shapes[i].cols ? 1 : 0;
-      m.tile_begin = tiles;
-      m.tiles_c = gp.np / kEwTileC;
-      m.ntiles = P.ew_ntiles[i];
-      m.scal_idx = P.scal_idx[i];
-      m.caller_idx = i;
-      m.part_begin = P.ew_part_begin[i];
-      m.nclusters = P.ew_nclusters[i];
-      tiles += P.ew_nclusters[i] * kEwCluster;
       const int vmul = (h->dtype == MUON_BF16) ? 8 : 4;
       if (!aligned16(m.src) || (m.mom && !aligned16(m.mom)) || (m.cols % vmul) != 0) vec_ok = 0;
     }
     prm.vec_ok = vec_ok;
-    prm.total_ctas = tiles;
     e = launch_momentum_norm(prm, io, xt, st);
     if (e != cudaSuccess) return e;
     ++*launches;
     trace(h, MUON_KERNEL_MOMENTUM_NORM, st);
   }
   return cudaSuccess;
+}
+
+// Tile tables of the single-launch schedule (everything but the tensor maps, pointers and
+// hyper-parameters): Update tiles 256 x 512 when every group's padded width allows it (except in
+// the iteration that writes W), Gram and Poly two upper blocks per tile, and the first tile of
+// each (stage, group) within an iteration.
+void fused_tables(const Plan& P, int nslots, int k, bool fuse_write, NsParams* q) {
+  std::memset(q, 0, sizeof(*q));
+  const int ng = static_cast<int>(P.groups.size());
+  bool wide = true;
+  for (const GroupPlan& gp : P.groups) wide = wide && gp.np % 512 == 0;
+  q->upd_tw[0] = wide ? 512 : 256;
+  q->upd_tw[1] = (wide && !fuse_write) ? 512 : 256;  // the Update that writes W keeps 256-wide tiles
+  q->sym_wide = 1;
+  for (int g = 0; g < ng; ++g) {
+    const GroupPlan& gp = P.groups[g];
+    NsGroup& G = q->g[g];
+    G.cnt = gp.cnt;
+    G.mp = gp.mp;
+    G.np = gp.np;
+    G.m_real = gp.m;
+    G.n_real = gp.n;
+    G.scal_base = gp.scal_base;
+    G.tdim = gp.mp / 256;
+  }
+  int iter_tiles[2] = {0, 0};
+  for (int L = 0; L < 2; ++L) {
+    int off = 0;
+    for (int kind = kGram; kind <= kUpdate; ++kind) {
+      for (int g = 0; g < ng; ++g) {
+        const GroupPlan& gp = P.groups[g];
+        const int T = gp.mp / 256;
+        const int tpm = kind == kUpdate ? T * (gp.np / q->upd_tw[L]) : sym_tiles(T, q->sym_wide != 0);
+        q->begin[L][kind][g] = off;
+        off += tpm * gp.cnt;
+      }
+      q->begin[L][kind][ng] = off;
+    }
+    iter_tiles[L] = off;
+  }
+  q->fuse_write = fuse_write ? 1 : 0;
+  q->ngroups = ng;
+  q->k = k;
+  q->nslots = nslots;
+  q->tiles_iter = k > 1 ? iter_tiles[0] : iter_tiles[1];
+  q->total_tiles = (k - 1) * iter_tiles[0] + iter_tiles[1];
 }
 
 // The parameter write can ride on the last Update launch when the parameters are bf16,
@@ -412,6 +491,68 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
   }
   const bool fuse = write_fusable(h, dst, k);
   *fused = fuse;
+  if (fused_schedule(h, k)) {
+    // every iteration in one launch: tiles of all 3k stages in one list, per-matrix counters
+    NvtxRange range("muon: Newton-Schulz, every iteration in one launch");
+    NsParams& q = h->ns;
+    fused_tables(P, h->n, k, fuse, &q);
+    const int ng = static_cast<int>(P.groups.size());
+    for (int g = 0; g < ng; ++g) {
+      const GroupPlan& gp = P.groups[g];
+      NsGroup& G = q.g[g];
+      for (int b = 0; b < 2; ++b) {
+        G.x_row[b] = gp.tm_x[b];
+        G.x_chk[b] = gp.tt_x[b];
+        G.x_st[b] = gp.ts_x[b];
+      }
+      G.a_row = gp.tm_a;
+      G.a_chk = gp.tt_a;
+      G.a_st = gp.ts_a;
+      G.b_row = gp.tm_b;
+      G.b_chk = gp.tt_b;
+      G.b_st = gp.ts_b;
+    }
+    q.a = hp->a;
+    q.b = hp->b;
+    q.c = hp->c;
+    q.scal = h->d_scal;
+    q.status = h->d_status;
+    q.deps = reinterpret_cast<unsigned int*>(h->ws + P.off_deps);
+    q.timeout_ns = kTimeoutNs;
+    if (fuse) {
+      q.w_decay = store_only ? 0.0f : 1.0f - hp->lr * hp->weight_decay;
+      for (const GroupPlan& gp : P.groups) {
+        for (int sl = 0; sl < gp.cnt; ++sl) {
+          const int i = gp.mats[sl], slot = gp.scal_base + sl;
+          const float r = static_cast<float>(h->shapes[i].rows), c = static_cast<float>(h->shapes[i].cols);
+          q.wptr[slot] = dst[i];
+          q.wcoef[slot] = store_only ? 1.0f : -hp->lr * std::sqrt(std::max(1.0f, r / c));
+          q.wtrans[slot] = h->shapes[i].rows > h->shapes[i].cols ? 1 : 0;
+        }
+      }
+    }
+    if (h->schedule != MUON_SCHEDULE_SPLIT) {
+      q.t_begin = 0;
+      q.t_end = q.total_tiles;
+      cudaError_t e = launch_ns_fused(q, h->num_sms, st);
+      if (e != cudaSuccess) return e;
+      ++*launches;
+      trace(h, MUON_KERNEL_NS_FUSED, st);
+      return cudaSuccess;
+    }
+    // the same tiles, one launch per stage (the stage boundaries then come from stream order)
+    for (int s = 0; s < 3 * k; ++s) {
+      const int it = s / 3, kind = s % 3, L = (it == k - 1) ? 1 : 0;
+      const int base = it * q.tiles_iter;
+      q.t_begin = base + q.begin[L][kind][0];
+      q.t_end = base + q.begin[L][kind][q.ngroups];
+      cudaError_t e = launch_ns_fused(q, h->num_sms, st);
+      if (e != cudaSuccess) return e;
+      ++*launches;
+      trace(h, MUON_KERNEL_GRAM + kind, st);
+    }
+    return cudaSuccess;
+  }
   for (int t = 1; t <= k; ++t) {
     const int cur = (t - 1) & 1, nxt = t & 1;
     if (h->mode == MUON_MODE_FAST) {
@@ -472,7 +613,6 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_bt = gp.tt_x[cur];
               G.tm_out = gp.ts_a;
               G.out = h->ws + gp.off_a;
-              G.aux = nullptr;
               G.tiles_per_mat = T * (T + 1) / 2;  // 256 x 256 pair tiles on or above the diagonal
               G.kblocks = gp.np / kTcBK;
               G.tdim = T;
@@ -485,7 +625,7 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_bt = gp.tt_a;
               G.tm_out = gp.ts_b;
               G.out = h->ws + gp.off_b;
-              G.aux = h->ws + gp.off_a;
+              G.tm_aux = gp.ts_a;
               G.tiles_per_mat = T * (T + 1) / 2;
               G.m_real = gp.m;
               G.kblocks = gp.mp / kTcBK;
@@ -498,7 +638,6 @@ cudaError_t enqueue_ns(muon_ctx* h, const muon_hparams_t* hp, cudaStream_t st, i
               G.tm_bt = gp.tt_x[cur];
               G.tm_out = gp.ts_x[nxt];
               G.out = h->ws + gp.off_x[nxt];
-              G.aux = nullptr;
               G.tiles_per_mat = (gp.mp / 256) * (gp.np / tw);  // 256 x tw pair tiles
               G.kblocks = gp.mp / kTcBK;
               G.tdim = gp.np / tw;
@@ -612,11 +751,14 @@ cudaError_t enqueue_back(muon_ctx* h, void* const* dst, const muon_hparams_t* hp
 
 int launches_for(const muon_ctx* h, int k) {
   const int chunks = (h->n + kEwMatsPerLaunch - 1) / kEwMatsPerLaunch;
-  if (small_path(h, k)) return chunks + 1 + chunks;
+  const int front = 2 * chunks;  // momentum/norm and the norms' finishing pass, per 192 matrices
+  if (small_path(h, k)) return front + 1 + chunks;
+  const bool fused_write = h->mode == MUON_MODE_FAST && h->dtype == MUON_BF16 && k >= 1 && h->fuse_shapes_ok;
+  if (fused_schedule(h, k))
+    return front + (h->schedule == MUON_SCHEDULE_SPLIT ? 3 * k : 1) + (fused_write ? 0 : chunks);
   const int ng = static_cast<int>(h->plan.groups.size());
   const int per_stage = (h->mode == MUON_MODE_FAST) ? (ng + kTcMaxGroups - 1) / kTcMaxGroups : ng;
-  const bool fused = h->mode == MUON_MODE_FAST && h->dtype == MUON_BF16 && k >= 1 && h->fuse_shapes_ok;
-  return chunks + 3 * k * per_stage + (fused ? 0 : chunks);
+  return front + 3 * k * per_stage + (fused_write ? 0 : chunks);
 }
 
 }  // namespace
@@ -683,7 +825,6 @@ muon_status_t muon_create(muon_handle_t* handle, const muon_shape_t* shapes, int
   h->ws = static_cast<char*>(workspace);
   h->ws_bytes = ws_bytes;
   h->d_status = reinterpret_cast<unsigned int*>(h->ws + h->plan.off_status);
-  h->d_counters = reinterpret_cast<unsigned int*>(h->ws + h->plan.off_counters);
   h->d_scal = reinterpret_cast<float*>(h->ws + h->plan.off_scal);
   h->d_partials = reinterpret_cast<float*>(h->ws + h->plan.off_partials);
   h->d_norms = reinterpret_cast<float*>(h->ws + h->plan.off_norms);
@@ -787,6 +928,48 @@ muon_status_t muon_get_plan(muon_handle_t h, int ns_steps, int* n_groups, int* l
   if (h == nullptr || ns_steps < 0 || ns_steps > 64) return MUON_ERR_INVALID_ARG;
   if (n_groups) *n_groups = static_cast<int>(h->plan.groups.size());
   if (launches_per_step) *launches_per_step = launches_for(h, ns_steps);
+  return MUON_OK;
+}
+
+muon_status_t muon_check_plan(const muon_shape_t* shapes, int n, int ns_steps, int num_sms, int64_t* problems) {
+  if (problems == nullptr || !shapes_ok(shapes, n) || ns_steps < 0 || ns_steps > 64 || num_sms < 2 ||
+      num_sms > kEwMaxCtas)
+    return MUON_ERR_INVALID_ARG;
+  Plan P;
+  make_plan(shapes, n, MUON_MODE_FAST, &P);
+  std::vector<muon_shape_t> sh(shapes, shapes + n);
+  long long bad = 0;
+  EwParams* ew = new (std::nothrow) EwParams;
+  NsParams* ns = new (std::nothrow) NsParams;
+  if (ew == nullptr || ns == nullptr) {
+    delete ew;
+    delete ns;
+    return MUON_ERR_INVALID_ARG;
+  }
+  for (int b = 0; b < n; b += kEwMatsPerLaunch) {
+    front_tables(P, sh, b, std::min(kEwMatsPerLaunch, n - b), num_sms, ew);
+    bad += check_front_tables(*ew);
+  }
+  if (ns_steps >= 1 && P.groups.size() <= static_cast<size_t>(kTcMaxGroups)) {
+    for (int fw = 0; fw < 2; ++fw) {
+      fused_tables(P, n, ns_steps, fw != 0, ns);
+      bad += check_fused_tiles(*ns);
+    }
+  }
+  delete ew;
+  delete ns;
+  *problems = bad;
+  return MUON_OK;
+}
+
+muon_status_t muon_set_schedule(muon_handle_t h, int schedule) {
+  if (h == nullptr) return MUON_ERR_INVALID_ARG;
+  if (schedule != MUON_SCHEDULE_AUTO && schedule != MUON_SCHEDULE_STAGED && schedule != MUON_SCHEDULE_FUSED &&
+      schedule != MUON_SCHEDULE_SPLIT)
+    return MUON_ERR_INVALID_ARG;
+  if ((schedule == MUON_SCHEDULE_FUSED || schedule == MUON_SCHEDULE_SPLIT) && !fused_possible(h, 1))
+    return MUON_ERR_UNSUPPORTED;
+  h->schedule = schedule;
   return MUON_OK;
 }
 

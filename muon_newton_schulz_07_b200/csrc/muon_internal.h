@@ -22,8 +22,8 @@ constexpr int kPad = 256;
 constexpr int kEwTileR = 64;
 constexpr int kEwTileC = 128;
 constexpr int kEwThreads = 256;
-constexpr int kEwCluster = 8;       // CTAs per cluster in the momentum/norm kernel
-constexpr int kEwTilesPerCta = 2;   // tiles per CTA in the momentum/norm kernel
+constexpr int kEwCtasPerSm = 2;     // resident CTAs per SM of the persistent momentum/norm kernel
+constexpr int kEwMaxCtas = 4096;    // upper bound of its grid (sizes the per-CTA partial sums)
 constexpr int kEwMatsPerLaunch = 192;
 
 enum Dtype : int { kBF16 = 0, kF32 = 1 };
@@ -35,26 +35,28 @@ struct EwMat {
   int rows, cols;    // caller's shape
   int mp, np;        // padded oriented shape
   int trans;         // rows > cols: X = U^T
-  int tile_begin;    // first CTA (cluster aligned) of this matrix in the launch
+  int tile_begin;    // first tile of this matrix in the launch's tile list
   int tiles_c;       // X tiles along np
-  int ntiles;        // X tiles of the padded matrix (mp/64 * np/128), kEwTilesPerCta per CTA
+  int ntiles;        // X tiles of the padded matrix (mp/64 * np/128)
   int scal_idx;      // slot of this matrix in the scalar / counter tables
   int caller_idx;    // position in the caller's matrix list
-  int part_begin;    // first per-cluster partial slot
-  int nclusters;     // clusters covering this matrix
+  int part_begin;    // first partial-sum slot of this matrix (a slot holds one sum per warp)
+  int nparts;        // CTAs that reach this matrix: min(ntiles, grid)
 };
 
+// The momentum/norm kernel is persistent: CTA c of a grid of P takes tiles c, c + P, c + 2P, ...
+// of the launch's T tiles (matrices back to back).
 struct EwParams {
   EwMat mat[kEwMatsPerLaunch];
   int nmat;
-  int total_ctas;
+  int total_tiles;
+  int grid;
   float beta;
   float eps;
   int nesterov;
   int vec_ok;              // every row of every matrix starts 16-byte aligned
-  float* partials;         // per-cluster sums of squares
+  float* partials;         // per (matrix, CTA, warp) sums of squares
   float* scal;             // per matrix: {||U||_F, 1/(||U||_F + eps)}
-  unsigned int* counters;  // per matrix arrival counters, zero before the launch
   float* norms;            // ||U||_F per matrix, caller order
 };
 
@@ -99,8 +101,8 @@ struct alignas(64) TcGroup {
   CUtensorMap tm_b;     // operand B source, row view
   CUtensorMap tm_bt;    // operand B source, chunked view
   CUtensorMap tm_out;   // output, store view: box 32 x 32 x 1, 64B swizzle
+  CUtensorMap tm_aux;   // Poly's epilogue input A, store view (box 32 x 32, 64B swizzle), loaded by TMA
   void* out;            // [cnt][rows][ld] bf16
-  const void* aux;      // [cnt][rows][ld] bf16 epilogue input, or nullptr
   int cnt, mp, np;
   int tiles_per_mat;
   int tile_begin;
@@ -142,6 +144,66 @@ struct TcParams {
 
 size_t tc_smem_bytes();
 cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s);
+
+// ------------------------------------------------------------------ every iteration in one launch
+// One persistent launch runs all k x {Gram, Poly, Update} stages of every matrix of up to
+// kTcMaxGroups shape groups.  Tiles are listed stage after stage (iteration-major, then
+// Gram / Poly / Update, then group, matrix and tile) and dealt round-robin to the CTA pairs;
+// before loading a tile, a pair waits (bounded) until the stage the tile reads is complete for
+// its matrix: every epilogue warp that finishes a tile adds 1 to a per (stage, matrix)
+// completion counter in the workspace.
+struct alignas(64) NsGroup {
+  CUtensorMap x_row[2], x_chk[2], x_st[2];  // X0 / X1: row, chunked and store views
+  CUtensorMap a_row, a_chk, a_st;           // A
+  CUtensorMap b_row, b_chk, b_st;           // B'
+  int cnt, mp, np;
+  int m_real, n_real;
+  int scal_base;        // first slot of the group in the scalar / counter tables
+  int tdim;             // mp / 256
+  int pad_[7];
+};
+
+struct NsParams {
+  NsGroup g[kTcMaxGroups];
+  int ngroups;
+  int k;                 // iterations, >= 1
+  int nslots;            // matrices of the launch (the counter table's row length)
+  int tiles_iter;        // tiles of an iteration other than the last
+  int total_tiles;
+  int t_begin, t_end;    // the tiles this launch runs: [0, total_tiles), or one stage of them
+  int upd_tw[2];         // Update tile width (256 or 512) of [other, last] iterations
+  int sym_wide;          // Gram and Poly take two neighbouring upper blocks per tile (256 x 512)
+  int fuse_write;        // the last Update writes the parameters (see TcParams)
+  // first tile of (stage, group) within an iteration, [other, last][stage][group];
+  // [..][stage][ngroups] is the end of the stage
+  int begin[2][3][kTcMaxGroups + 1];
+  float a, b, c;
+  const float* scal;
+  unsigned int* status;
+  unsigned int* deps;    // [3 k][nslots] completion counters, zero before the launch
+  unsigned long long timeout_ns;
+  float w_decay;
+  void* wptr[kTcMaxFused];
+  float wcoef[kTcMaxFused];
+  unsigned char wtrans[kTcMaxFused];
+};
+
+// Tiles per matrix of a symmetric stage (Gram, Poly) over the T x T blocks of the upper
+// triangle: one per block, or (wide) one per pair of neighbouring blocks of a block row, with a
+// 256-wide tile for the odd block at the end of a row.
+__host__ __device__ inline int sym_tiles(int T, bool wide) {
+  if (!wide) return T * (T + 1) / 2;
+  int n = 0;
+  for (int I = 0; I < T; ++I) n += (T - I + 1) / 2;
+  return n;
+}
+
+size_t fused_smem_bytes();
+cudaError_t launch_ns_fused(const NsParams& p, int num_sms, cudaStream_t s);
+// Host-side consistency check of a single-launch tile list (number of problems found).
+long long check_fused_tiles(const NsParams& p);
+// Host-side consistency check of one momentum/norm launch's tables (number of problems found).
+long long check_front_tables(const EwParams& p);
 
 // ------------------------------------------------------------------ small matrices, all iterations in one kernel
 // Every matrix of the set fits one 256 x 256 tile (max(rows, cols) <= 256; the workspace

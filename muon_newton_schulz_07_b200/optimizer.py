@@ -18,7 +18,10 @@ QUINTIC = (3.4445, -4.7750, 2.0315)
 class MuonStep:
     """A Muon step for one fixed list of matrix shapes, bound to one CUDA device."""
 
-    def __init__(self, shapes, dtype=torch.bfloat16, mode: str = "fast", device=None):
+    SCHEDULES = {"auto": B.MUON_SCHEDULE_AUTO, "staged": B.MUON_SCHEDULE_STAGED, "fused": B.MUON_SCHEDULE_FUSED,
+                 "split": B.MUON_SCHEDULE_SPLIT}
+
+    def __init__(self, shapes, dtype=torch.bfloat16, mode: str = "fast", device=None, schedule: str = "auto"):
         if dtype not in (torch.bfloat16, torch.float32):
             raise TypeError("dtype must be torch.bfloat16 or torch.float32")
         if mode not in ("fast", "fp32_ref"):
@@ -36,6 +39,15 @@ class MuonStep:
             self._ws_ptr = (base + 1023) // 1024 * 1024
             self.handle = B.muon_create(self.shapes, self._dt, self._mode, self._ws_ptr, nbytes)
         self.n_groups, _ = B.muon_get_plan(self.handle, 5)
+        if schedule != "auto":
+            self.set_schedule(schedule)
+
+    def set_schedule(self, schedule: str) -> None:
+        """'auto', 'staged' (one launch per Newton-Schulz stage), 'fused' (every iteration in one launch)
+        or 'split' (the fused kernel's tiles, one launch per stage)."""
+        if schedule not in self.SCHEDULES:
+            raise ValueError(f"schedule must be one of {sorted(self.SCHEDULES)}")
+        B.muon_set_schedule(self.handle, self.SCHEDULES[schedule])
 
     def launches_per_step(self, ns_steps: int = 5) -> int:
         return B.muon_get_plan(self.handle, ns_steps)[1]

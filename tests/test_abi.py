@@ -107,3 +107,24 @@ def test_adamw_arguments_checked_on_host():
     with pytest.raises(B.MuonError):
         B.muon_adamw_step([16], [16], [16], [16], [-1], B.MUON_BF16, ok, 0)
     assert lib is not None
+
+
+@pytest.mark.parametrize("num_sms", [148, 132, 8])
+@pytest.mark.parametrize("k", [1, 2, 5, 10])
+@pytest.mark.parametrize("name", ["d24", "gpt2s", "l38b", "stress", "single256"])
+def test_launch_tables_are_consistent(name, k, num_sms):
+    # the host-built tables of the persistent momentum/norm kernel and of the single-launch
+    # Newton-Schulz schedule, checked by the library itself (no device needed)
+    shapes = list(I.WORKLOADS[name].shapes)
+    assert B.muon_check_plan(shapes, k, num_sms) == 0
+
+
+@pytest.mark.parametrize("shapes", [
+    [(200, 328), (328, 200), (520, 1000), (300, 300)],
+    [(256, 512), (512, 768), (768, 1024), (1024, 256), (300, 1300), (512, 512)],
+    [(8, 8), (1, 300), (300, 1), (130, 130)],
+    [(1536, 1536)] * 200 + [(256, 4096)] * 3,
+])
+def test_launch_tables_ragged_and_many(shapes):
+    for k in (1, 3, 5):
+        assert B.muon_check_plan(shapes, k, 148) == 0

@@ -35,20 +35,24 @@ def test_byte_counts_per_element():
 
 
 def test_traffic_record_is_used_only_for_the_captured_source(tmp_path, monkeypatch):
-    rec_path = os.path.join(bench.ROOT, "profiles", "traffic_update_d24.json")
-    with open(rec_path) as f:
-        rec = json.load(f)
-    got = bench.measured_traffic("update", "d24")
-    assert got == (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * rec["scale_to_workload"]["d24"]
+    import hashlib
+
+    # a record of a capture, and the kernel source it was taken from
+    root = tmp_path / "repo"
+    (root / "profiles").mkdir(parents=True)
+    src = root / "csrc" / "kernel.cu"
+    src.parent.mkdir(parents=True)
+    src.write_text("// the captured kernel\n")
+    rec = {"kernel": "k", "source": "csrc/kernel.cu",
+           "source_sha256_16": hashlib.sha256(src.read_bytes()).hexdigest()[:16],
+           "dram_bytes_read": 600.0, "dram_bytes_write": 400.0, "scale_to_workload": {"d24": 3.0}}
+    (root / "profiles" / "traffic_update_d24.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.measured_traffic("update", "d24") == 3000.0
     assert bench.measured_traffic("update", "gpt2s") is None  # no capture for that workload
     assert bench.measured_traffic("gram", "d24") is None      # no record for that kernel
     # a changed kernel source invalidates the record
-    root = tmp_path / "repo"
-    shutil.copytree(os.path.join(bench.ROOT, "profiles"), root / "profiles")
-    src = root / rec["source"]
-    src.parent.mkdir(parents=True)
     src.write_text("// a different kernel\n")
-    monkeypatch.setattr(bench, "ROOT", str(root))
     assert bench.measured_traffic("update", "d24") is None
 
 

@@ -9,6 +9,9 @@ Tolerances (relative Frobenius error, max over matrices):
     spacing) and carries lr*s times the error of O, so
     ||W1 - W1_ref||_F <= 0.5 ||ulp(W1_ref)||_F * 1.01 + lr * s * 2e-2 * ||O_ref||_F.
     In fp32 storage (W1 - W)/(-lr*s) is O itself and is checked at O's tolerance.
+Element by element, M1 lies within half a storage spacing of the oracle's value, and W1 within
+half a spacing plus the direction error of that element (a second step from W = 0 stores the
+direction the step applied; see helpers.assert_w1_elementwise).
 """
 from __future__ import annotations
 
@@ -23,7 +26,8 @@ from muon_newton_schulz_07_b200 import binding as B
 from muon_newton_schulz_07_b200 import inputs as I
 from muon_newton_schulz_07_b200.optimizer import MuonStep
 
-from helpers import bf16_ulp, device_tensor, rel_fro, to_f64, workload_tensors
+from helpers import (assert_m1_elementwise, assert_w1_elementwise, bf16_ulp, device_tensor, rel_fro,
+                     step_with_direction, to_f64, workload_tensors)
 
 pytestmark = pytest.mark.gpu
 
@@ -52,11 +56,13 @@ def test_single256_step(mode):
     W, G, M = workload_tensors(wl, torch.float32)
     W0, G0, M0 = to_f64(W[0]), to_f64(G[0]), to_f64(M[0])
     op = MuonStep(wl.shapes, dtype=torch.float32, mode=mode)
-    op(W, G, M, lr=0.02, beta=0.95, weight_decay=0.0, ns_steps=5)
-    torch.cuda.synchronize()
+    Wz = step_with_direction(op, W, G, M, lr=0.02, beta=0.95, weight_decay=0.0, ns_steps=5)
     assert op.status() == B.MUON_OK
     W1r, M1r, Or = O.muon_step(W0, G0, M0, oracle_hp())
     assert rel_fro(to_f64(M[0]), M1r) < 2.0 ** -23
+    assert_m1_elementwise(to_f64(M[0]), M1r, M0, G0, torch.float32)
+    Wzr = O.parameter_write(np.zeros_like(W0), Or, 0.02, 0.0)
+    assert_w1_elementwise(to_f64(W[0]), W1r, to_f64(Wz[0]), Wzr, W0, torch.float32)
     O_gpu = (to_f64(W[0]) - W0) / (-0.02 * O.shape_scale(256, 256))
     err = rel_fro(O_gpu, Or)
     print(f"single256 {mode}: O rel err {err:.3e}")
@@ -217,16 +223,20 @@ def test_gpt2s_steps_teacher_forced():
         if step > 1:
             G = [device_tensor(I.gradient(wl, step, i), torch.bfloat16) for i in range(len(wl.shapes))]
         pre = {i: (to_f64(W[i]), to_f64(G[i]), to_f64(M[i])) for i in check}
-        op(W, G, M, lr=0.02, beta=0.95, ns_steps=5)
-        torch.cuda.synchronize()
+        Wz = step_with_direction(op, W, G, M, lr=0.02, beta=0.95, ns_steps=5)
         assert op.status() == B.MUON_OK
         for i in check:
             W0, G0, M0 = pre[i]
             W1r, M1r, Or = O.muon_step(W0, G0, M0, oracle_hp())
             assert rel_fro(to_f64(M[i]), M1r) < 2.0 ** -8
+            assert_m1_elementwise(to_f64(M[i]), M1r, M0, G0, torch.bfloat16, what=f"M1 step {step} matrix {i}")
             r, c = wl.shapes[i]
             bound = 0.5 * 1.01 * np.linalg.norm(bf16_ulp(W1r)) + 0.02 * O.shape_scale(r, c) * 2e-2 * np.linalg.norm(Or)
             assert np.linalg.norm(to_f64(W[i]) - W1r) <= bound, (step, i)
+            Wzr = O.parameter_write(np.zeros_like(W0), Or, 0.02, 0.0)
+            assert rel_fro(to_f64(Wz[i]), Wzr) < 2e-2 + 2.0 ** -8, (step, i)
+            assert_w1_elementwise(to_f64(W[i]), W1r, to_f64(Wz[i]), Wzr, W0, torch.bfloat16,
+                                  what=f"W1 step {step} matrix {i}")
 
 
 def test_gpt2s_orthogonal_direction():
