@@ -46,6 +46,8 @@ def parse():
                     help="use only the first N matrices of the workload (profiling captures of a smaller case)")
     ap.add_argument("--schedule", choices=["auto", "staged", "fused", "split"], default="auto",
                     help="Newton-Schulz launch schedule of the library (staged: one launch per stage)")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of CUDA graphs of the step (captured through the C ABI) instead of eager calls")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-adamw", action="store_true", help="skip the AdamW leg (non-matrix parameters)")
@@ -377,10 +379,17 @@ def torch_from(a, dev, dt):
     return torch.from_numpy(a).to(dev).to(dt)
 
 
-def timed_steps(step_fn, G_sets, steps, warmup, op, dev, stream, local_rank, sync_all, in_bytes, B):
-    """W warm-up steps, then `steps` timed steps with CUDA events on the launching stream and the
-    library's per-kernel tracing; clocks sampled meanwhile.  Inputs smaller than L2 get a 512 MB
-    scratch write before every timed step (outside that step's events)."""
+def timed_steps(step_fn, G_sets, steps, warmup, op, dev, stream, local_rank, sync_all, in_bytes, B, graph=False):
+    """W warm-up steps, then `steps` timed steps with CUDA events on the launching stream; clocks
+    sampled meanwhile.  Inputs smaller than L2 get a 512 MB scratch write before every timed step
+    (outside that step's events).
+
+    Eager: the timed steps also carry the library's per-kernel tracing.  Graph: one step per
+    gradient set is captured into a CUDA graph (the library's muon_step is capturable) and the
+    timed steps replay them, which removes the host's per-launch cost and the gaps between
+    launches; the per-kernel times then come from a separate traced eager pass of the same
+    steps.  Returns (ms_total, per-kernel profile, clocks, flushed, eager ms per step or None).
+    """
     import torch
 
     for i in range(warmup):
@@ -388,17 +397,38 @@ def timed_steps(step_fn, G_sets, steps, warmup, op, dev, stream, local_rank, syn
     sync_all()
     if op.status() != B.MUON_OK:
         raise RuntimeError("device status after warm-up is not OK")
+    graphs = None
+    if graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        graphs = [torch.cuda.CUDAGraph() for _ in range(2)]
+        with torch.cuda.stream(side):
+            for i in range(2):
+                with torch.cuda.graph(graphs[i], stream=side):
+                    step_fn(G_sets[i])
+        stream.wait_stream(side)
+        for i in range(2):  # a replay of each before timing
+            graphs[i].replay()
+        sync_all()
+
+    def one(i):
+        if graphs is not None:
+            graphs[i % 2].replay()
+        else:
+            step_fn(G_sets[i % 2])
+
     clocks = ClockSampler(gpu_index_for(local_rank))
     clocks.start()
     time.sleep(0.3)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if in_bytes < L2_FLUSH_BELOW else None
-    B.muon_profile_begin(op.handle, steps)
+    if graphs is None:
+        B.muon_profile_begin(op.handle, steps)
     sync_all()
     if flush is None:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for i in range(steps):
-            step_fn(G_sets[i % 2])
+            one(i)
         e1.record(stream)
         sync_all()
         ms_total = e0.elapsed_time(e1)
@@ -407,16 +437,30 @@ def timed_steps(step_fn, G_sets, steps, warmup, op, dev, stream, local_rank, syn
         for i in range(steps):
             flush.fill_(i & 0xFF)
             ev[i][0].record(stream)
-            step_fn(G_sets[i % 2])
+            one(i)
             ev[i][1].record(stream)
         sync_all()
         ms_total = sum(a.elapsed_time(b) for a, b in ev)
     clk = clocks.stop()
-    prof = B.muon_profile_end(op.handle)
+    eager_ms = None
+    if graphs is None:
+        prof = B.muon_profile_end(op.handle)
+    else:
+        # per-kernel times from a traced eager pass (same steps, outside the timed region)
+        B.muon_profile_begin(op.handle, steps)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            step_fn(G_sets[i % 2])
+        e1.record(stream)
+        sync_all()
+        prof = B.muon_profile_end(op.handle)
+        eager_ms = e0.elapsed_time(e1) / steps
+        del graphs
     status = op.status()
     if status != B.MUON_OK:
         raise RuntimeError(f"device status after the timed steps: {B.STATUS.get(status, status)}")
-    return ms_total, prof, clk, flush is not None
+    return ms_total, prof, clk, flush is not None, eager_ms
 
 
 # Further workloads timed after the headline one (one GPU only), each its own block of the line.
@@ -428,7 +472,7 @@ EXTRA_LEGS = {
 }
 
 
-def run_extra_leg(leg, warmup, dev, local_rank, peaks, peak_src, schedule="auto", cache=None):
+def run_extra_leg(leg, warmup, dev, local_rank, peaks, peak_src, schedule="auto", cache=None, graph=False):
     """One further workload leg; `cache` keeps the last workload's inputs for the next leg."""
     import torch
 
@@ -458,8 +502,8 @@ def run_extra_leg(leg, warmup, dev, local_rank, peaks, peak_src, schedule="auto"
         op(W, Gs, M, ns_steps=k)
 
     in_bytes = sum(t.numel() * t.element_size() for t in list(W) + list(M) + list(G_sets[0]))
-    ms_total, prof, clk, flushed = timed_steps(step_fn, G_sets, steps, warmup, op, dev, stream, local_rank,
-                                               lambda: torch.cuda.synchronize(dev), in_bytes, B)
+    ms_total, prof, clk, flushed, eager_ms = timed_steps(step_fn, G_sets, steps, warmup, op, dev, stream, local_rank,
+                                                         lambda: torch.cuda.synchronize(dev), in_bytes, B, graph)
     kern, roof, ns, targets = kernel_table(prof, shapes, k, 4 if dt == torch.float32 else 2, steps, peaks, peak_src,
                                            wl.name)
     ms = ms_total / steps
@@ -468,7 +512,8 @@ def run_extra_leg(leg, warmup, dev, local_rank, peaks, peak_src, schedule="auto"
            "roofline": roof, "ns": ns, "kernels": kern, "targets": targets,
            "gpu_launches": op.launches_per_step(k) * steps, "clocks": clk,
            "l2": "flushed before every timed step" if flushed else "inputs larger than L2, no flush",
-           "input_generation_s": gen_s}
+           "input_generation_s": gen_s, "launch": "cuda graph replay" if graph else "eager",
+           "eager_ms_per_step": eager_ms}
     op.close()
     del W, M, G_sets
     if cache is None:
@@ -535,8 +580,9 @@ def run_muon(args, rank, world, local_rank):
         return float(t.item())
 
     in_bytes = sum(t.numel() * t.element_size() for t in list(W) + list(M) + list(G_sets[0]))
-    ms_total, prof, clk, flushed = timed_steps(step_fn, G_sets, args.steps, args.warmup, op, dev, stream, local_rank,
-                                               sync_all, in_bytes, B)
+    ms_total, prof, clk, flushed, eager_ms = timed_steps(step_fn, G_sets, args.steps, args.warmup, op, dev, stream,
+                                                         local_rank, sync_all, in_bytes, B,
+                                                         args.graph and not sharded)
     ms_per_step = max_over_ranks(ms_total / args.steps)
     value = (1 if sharded else world) * 1000.0 / ms_per_step
 
@@ -633,7 +679,8 @@ def run_muon(args, rank, world, local_rank):
         extra = {}
         cache = {}
         for leg in [x for x in args.extra.split(",") if x]:
-            extra[leg] = run_extra_leg(leg, args.warmup, dev, local_rank, peaks, peak_src, args.schedule, cache)
+            extra[leg] = run_extra_leg(leg, args.warmup, dev, local_rank, peaks, peak_src, args.schedule, cache,
+                                       args.graph)
         cache.clear()
         torch.cuda.empty_cache()
 
@@ -661,6 +708,8 @@ def run_muon(args, rank, world, local_rank):
             "e2e": e2e,
             "gpu_launches": launches * args.steps,
             "clocks": clk,
+            "launch": "cuda graph replay" if (args.graph and not sharded) else "eager",
+            "eager_ms_per_step": eager_ms,
         }
         if extra is not None:
             line["workloads"] = extra

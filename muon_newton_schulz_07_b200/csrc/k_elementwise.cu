@@ -27,6 +27,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <vector>
 
 #include "muon_device.cuh"
@@ -174,13 +175,22 @@ __device__ __forceinline__ void momentum_chunk(const EwMat& mt, const EwParams& 
     float g[8];
     c.g[q].to_f32x8(g);
     if (mom != nullptr) {
+      // the same fp32 products and fused multiply-adds as the scalar path, two lanes per
+      // instruction (f32x2: each lane rounds exactly like fmaf / a * b)
       float m[8];
       c.m[q].to_f32x8(m);
+      const float2 b2 = make_float2(beta, beta), o2 = make_float2(omb, omb);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m[i] = fmaf(beta, m[i], omb * g[i]);
+      for (int i = 0; i < 8; i += 2) {
+        const float2 og = __fmul2_rn(o2, make_float2(g[i], g[i + 1]));
+        const float2 m1 = __ffma2_rn(b2, make_float2(m[i], m[i + 1]), og);
+        const float2 u1 = p.nesterov ? __ffma2_rn(b2, m1, og) : m1;
+        m[i] = m1.x;
+        m[i + 1] = m1.y;
+        u[i] = u1.x;
+        u[i + 1] = u1.y;
+      }
       Raw8<T>::store_cs(mom + base, m);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) u[i] = p.nesterov ? fmaf(beta, m[i], omb * g[i]) : m[i];
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) u[i] = g[i];
@@ -223,7 +233,17 @@ __device__ __forceinline__ void momentum_tile_load(const EwMat& mt, const EwPara
 
 // The rest of the tile once its loads are in `ch`: momentum/Nesterov, M1 stored, U stored to X0
 // (transposed through shared memory for tall matrices); returns this thread's sum of squares.
-template <typename T, typename XT, int LD>
+// A barrier over the kEwThreads threads that compute (named barrier 1: the bulk-copy kernel's
+// producer warp does not take part), or the whole CTA.
+template <bool NAMED>
+__device__ __forceinline__ void compute_sync() {
+  if (NAMED)
+    asm volatile("bar.sync 1, %0;" ::"n"(kEwThreads) : "memory");
+  else
+    __syncthreads();
+}
+
+template <typename T, typename XT, int LD, bool NAMED = false>
 __device__ __forceinline__ float momentum_tile_store(const EwMat& mt, const EwParams& p, int t,
                                                      const MomentumChunks<T>& ch, XT (*stage)[LD]) {
   float ss = 0.0f;
@@ -240,7 +260,7 @@ __device__ __forceinline__ float momentum_tile_store(const EwMat& mt, const EwPa
       Vec8<XT>::store(x + static_cast<size_t>(xr0 + r) * mt.np + xc0 + cc, u);
     }
   } else {
-    __syncthreads();  // the previous tile's staged values have been read out
+    compute_sync<NAMED>();  // the previous tile's staged values have been read out
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int c = threadIdx.x + q * kEwThreads;
@@ -250,7 +270,7 @@ __device__ __forceinline__ float momentum_tile_store(const EwMat& mt, const EwPa
 #pragma unroll
       for (int i = 0; i < 8; ++i) stage[sc + i][sr] = from_f32<XT>(u[i]);
     }
-    __syncthreads();
+    compute_sync<NAMED>();
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int c = threadIdx.x + q * kEwThreads;
@@ -337,6 +357,141 @@ __global__ void __launch_bounds__(kEwThreads, kEwCtasPerSm) momentum_norm_kernel
     }
   }
   momentum_flush(p, p.mat[mi], ss);
+}
+
+// ---------------------------------------------------------------- async-copy-fed variant
+// For launches whose sources are 16-byte aligned with rows a multiple of 8 elements (vec_ok): one
+// CTA of 256 threads per SM, each thread streaming its own 16-byte pieces of G and M for the next
+// kAsyncStages - 1 tiles into shared memory with cp.async (no registers held for data in flight),
+// then computing a tile from its own pieces.  Five tiles (160 KB for bf16) are in flight per SM.
+template <typename T> struct AsyncGeometry {
+  static constexpr int STAGE = 2 * kEwTileR * kEwTileC * static_cast<int>(sizeof(T));  // G and M of one tile
+  static constexpr int STAGES = sizeof(T) == 2 ? 5 : 3;
+};
+
+template <typename T, typename XT>
+size_t async_smem_bytes() {
+  constexpr int LD = kEwTileC + (sizeof(XT) == 2 ? 2 : 1);
+  return static_cast<size_t>(AsyncGeometry<T>::STAGES) * AsyncGeometry<T>::STAGE +
+         static_cast<size_t>(kEwTileR) * LD * sizeof(XT);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// The 16-byte pieces of tile t (matrix mt) this thread works on, G and M, into its slots of one
+// stage: piece (q, which) of thread i sits at ((which * 4 + q) * kEwThreads + i) pieces from the
+// stage's start, so neighbouring threads touch neighbouring 16 bytes.  Pieces outside the matrix
+// are not copied (momentum_chunk gives them U = 0 without reading).
+template <typename T>
+__device__ __forceinline__ void momentum_tile_async(const EwMat& mt, int t, uint32_t stage) {
+  constexpr int PIECE = 16;
+  constexpr int PER8 = static_cast<int>(sizeof(T)) * 8 / PIECE;  // 16-byte pieces per 8 elements
+  const int xr0 = (t / mt.tiles_c) * kEwTileR;
+  const int xc0 = (t % mt.tiles_c) * kEwTileC;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = threadIdx.x + q * kEwThreads;
+    const int row = mt.trans ? xc0 + (c >> 3) : xr0 + (c >> 4);
+    const int col = mt.trans ? xr0 + (c & 7) * 8 : xc0 + (c & 15) * 8;
+    if (row < mt.rows && col + 8 <= mt.cols) {
+      const size_t base = static_cast<size_t>(row) * mt.cols + col;
+#pragma unroll
+      for (int h = 0; h < PER8; ++h) {
+        const uint32_t off = static_cast<uint32_t>(((0 * 4 + q) * PER8 + h) * kEwThreads + threadIdx.x) * PIECE;
+        cp_async16(stage + off, static_cast<const T*>(mt.src) + base + h * (8 / PER8));
+        if (mt.mom != nullptr) {
+          const uint32_t offm = static_cast<uint32_t>(((1 * 4 + q) * PER8 + h) * kEwThreads + threadIdx.x) * PIECE;
+          cp_async16(stage + offm, static_cast<const T*>(mt.mom) + base + h * (8 / PER8));
+        }
+      }
+    }
+  }
+}
+
+// The pieces of tile t this thread copied into stage `st`, as MomentumChunks.
+template <typename T>
+__device__ __forceinline__ void momentum_tile_from_async(const EwMat& mt, int t, const uint8_t* st,
+                                                         MomentumChunks<T>& c) {
+  constexpr int PIECE = 16;
+  constexpr int PER8 = static_cast<int>(sizeof(T)) * 8 / PIECE;
+  const int xr0 = (t / mt.tiles_c) * kEwTileR;
+  const int xc0 = (t % mt.tiles_c) * kEwTileC;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int cc = threadIdx.x + q * kEwThreads;
+    const int row = mt.trans ? xc0 + (cc >> 3) : xr0 + (cc >> 4);
+    const int col = mt.trans ? xr0 + (cc & 7) * 8 : xc0 + (cc & 15) * 8;
+    c.vec[q] = row < mt.rows && col + 8 <= mt.cols;
+    if (c.vec[q]) {
+#pragma unroll
+      for (int h = 0; h < PER8; ++h) {
+        reinterpret_cast<uint4*>(&c.g[q])[h] =
+            *reinterpret_cast<const uint4*>(st + (((0 * 4 + q) * PER8 + h) * kEwThreads + threadIdx.x) * PIECE);
+        if (mt.mom != nullptr)
+          reinterpret_cast<uint4*>(&c.m[q])[h] =
+              *reinterpret_cast<const uint4*>(st + (((1 * 4 + q) * PER8 + h) * kEwThreads + threadIdx.x) * PIECE);
+      }
+    }
+  }
+}
+
+template <typename T, typename XT>
+__global__ void __launch_bounds__(kEwThreads, 1) momentum_norm_async_kernel(const __grid_constant__ EwParams p) {
+  constexpr int LD = kEwTileC + (sizeof(XT) == 2 ? 2 : 1);
+  constexpr int NS = AsyncGeometry<T>::STAGES;
+  constexpr int SB = AsyncGeometry<T>::STAGE;
+  extern __shared__ __align__(16) uint8_t smem_async[];
+  XT(*stage)[LD] = reinterpret_cast<XT(*)[LD]>(smem_async + NS * SB);
+  const uint32_t ring = smem_u32(smem_async);
+  const int step = static_cast<int>(gridDim.x);
+  const int t0 = static_cast<int>(blockIdx.x);
+  if (t0 >= p.total_tiles) return;
+  int lo = 0, hi = p.nmat - 1;  // matrix of t0
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.mat[mid].tile_begin <= t0) lo = mid; else hi = mid - 1;
+  }
+  // prologue: the first NS - 1 tiles of this CTA on their way (one copy group per tile)
+  int mload = lo;
+#pragma unroll 1
+  for (int k = 0; k < NS - 1; ++k) {
+    const int t = t0 + k * step;
+    if (t < p.total_tiles) {
+      mload = matrix_of_tile(p, mload, t);
+      momentum_tile_async<T>(p.mat[mload], t - p.mat[mload].tile_begin, ring + k * SB);
+    }
+    cp_async_commit();
+  }
+  int mi = lo, macc = lo, j = 0;
+  float ss = 0.0f;
+#pragma unroll 1
+  for (int t = t0; t < p.total_tiles; t += step, ++j) {
+    // the tile NS - 1 ahead into the slot the previous iteration has finished reading
+    const int tn = t + (NS - 1) * step;
+    if (tn < p.total_tiles) {
+      mload = matrix_of_tile(p, mload, tn);
+      momentum_tile_async<T>(p.mat[mload], tn - p.mat[mload].tile_begin, ring + ((j + NS - 1) % NS) * SB);
+    }
+    cp_async_commit();
+    cp_async_wait<NS - 1>();   // this thread's pieces of tile t have landed
+    mi = matrix_of_tile(p, mi, t);
+    const EwMat& mt = p.mat[mi];
+    MomentumChunks<T> ch;
+    momentum_tile_from_async<T>(mt, t - mt.tile_begin, smem_async + (j % NS) * SB, ch);
+    if (mi != macc) {
+      momentum_flush(p, p.mat[macc], ss);
+      ss = 0.0f;
+      macc = mi;
+    }
+    ss += momentum_tile_store<T, XT, LD>(mt, p, t - mt.tile_begin, ch, stage);
+  }
+  cp_async_wait<0>();
+  momentum_flush(p, p.mat[macc], ss);
 }
 
 // The norms of one momentum/norm launch's matrices: CTA j adds matrix j's per-warp partial sums
@@ -465,8 +620,26 @@ __global__ void __launch_bounds__(kEwThreads, 3) param_write_kernel(const __grid
 
 template <typename T, typename XT>
 cudaError_t launch_mn(const EwParams& p, cudaStream_t s) {
-  momentum_norm_kernel<T, XT><<<p.grid, kEwThreads, 0, s>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (p.vec_ok) {
+    // async-copy-fed: one CTA per SM (the tables were built for that grid)
+    static std::atomic<unsigned long long> attr_set{0};
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    const size_t smem = async_smem_bytes<T, XT>();
+    if ((attr_set.load() & bit) == 0) {
+      e = cudaFuncSetAttribute(momentum_norm_async_kernel<T, XT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      attr_set.fetch_or(bit);
+    }
+    momentum_norm_async_kernel<T, XT><<<p.grid, kEwThreads, smem, s>>>(p);
+  } else {
+    momentum_norm_kernel<T, XT><<<p.grid, kEwThreads, 0, s>>>(p);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   norm_finish_kernel<<<p.nmat, kEwThreads, 0, s>>>(p);
   return cudaGetLastError();

@@ -45,26 +45,36 @@ namespace {
 
 constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK;
 constexpr int TILE = 256;
-constexpr int NST = 3;                              // operand ring stages
 constexpr uint32_t A_STAGE = BM * BK * 2;           // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t B_STAGE = (BN / 2) * BK * 2;     // 16 KB: this CTA's half of one 256-column B tile
-constexpr uint32_t SB = A_STAGE + 2 * B_STAGE;      // 48 KB: room for the operands of a 512-wide tile
 constexpr uint32_t TMEM_COLS = 512;                 // two 256-column accumulator slots
 constexpr int EPI_WARPS = kTcEpiWarps;
 constexpr int F32_PITCH = 36;                        // staged fp32 row: 32 + 4 pad
-constexpr uint32_t STAGE_REGION = NST * SB;
 constexpr uint32_t EPI_OUT_BYTES = 2048;
 constexpr uint32_t EPI_AUX_BYTES = 2048;              // one 32 x 32 bf16 chunk of A (64B swizzle)
 constexpr uint32_t EPI_F32_BYTES = 32 * F32_PITCH * 4;
-constexpr uint32_t EPI_OFFSET = STAGE_REGION;
-constexpr uint32_t EPI_AUX_OFFSET = EPI_OFFSET + EPI_WARPS * 2 * EPI_OUT_BYTES;
-constexpr uint32_t BAR_OFFSET = EPI_AUX_OFFSET + EPI_WARPS * 2 * EPI_AUX_BYTES;
 constexpr uint32_t BAR_BYTES = 256;
-constexpr size_t SMEM_BYTES = 1024 + BAR_OFFSET + BAR_BYTES;
+
+// The operand ring: stages of 48 KB (three) when the list holds 512-wide tiles, else stages of
+// 32 KB (five), after which come the epilogue's store tiles and A chunks and the barriers.
+template <bool WR>
+struct FLayout {
+  static constexpr int NST = WR ? 3 : 5;
+  static constexpr uint32_t SB = A_STAGE + (WR ? 2 : 1) * B_STAGE;
+  // Each epilogue warp owns one 8 KB block: its two store tiles, then its two A chunks.  The
+  // fp32 staging of the fused parameter write overlays the warp's own block only (a warp on a
+  // parameter-writing tile has no store or A load of its own in flight), never another warp's:
+  // the warps of a pair drift apart by up to two tiles, and a neighbour may still be reading
+  // its A chunks of an earlier polynomial tile.
+  static constexpr uint32_t EPI_OFFSET = NST * SB;
+  static constexpr uint32_t EPI_WARP_BYTES = 2 * EPI_OUT_BYTES + 2 * EPI_AUX_BYTES;
+  static constexpr uint32_t BAR_OFFSET = EPI_OFFSET + EPI_WARPS * EPI_WARP_BYTES;
+  static constexpr size_t SMEM_BYTES = 1024 + BAR_OFFSET + BAR_BYTES;
+  static_assert(EPI_F32_BYTES <= EPI_WARP_BYTES, "fp32 staging must fit the warp's own block");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(2 * NST + 5 + 2 * EPI_WARPS <= BAR_BYTES / 8, "barriers must fit their region");
+};
 constexpr unsigned int ARRIVALS_PER_TILE = 2 * EPI_WARPS;   // epilogue warps of both CTAs
-static_assert(EPI_WARPS * EPI_F32_BYTES <= BAR_OFFSET - EPI_OFFSET, "fp32 staging must fit the epilogue region");
-static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-static_assert(2 * NST + 5 + 2 * EPI_WARPS <= BAR_BYTES / 8, "barriers must fit their region");
 static_assert(sizeof(NsParams) <= 32764, "kernel parameters are limited to 32764 bytes");
 
 struct FTile {
@@ -194,8 +204,13 @@ __device__ __forceinline__ void mma_slice(uint32_t d_tmem, uint32_t sa, uint32_t
     tc_mma_bf16_pair(d_tmem, adesc0 + astep * j, bdesc0 + bstep * j, idesc, (!first || j != 0) ? 1u : 0u);
 }
 
+template <bool WR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     ns_fused_kernel(const __grid_constant__ NsParams p) {
+  constexpr int NST = FLayout<WR>::NST;
+  constexpr uint32_t SB = FLayout<WR>::SB;
+  constexpr uint32_t EPI_OFFSET = FLayout<WR>::EPI_OFFSET, EPI_WARP_BYTES = FLayout<WR>::EPI_WARP_BYTES,
+                     BAR_OFFSET = FLayout<WR>::BAR_OFFSET;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t smem_base = smem_u32(smem);
@@ -275,6 +290,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         const CUtensorMap* mb_chk = f.kind == kGram ? &G.x_chk[cur] : f.kind == kPoly ? &G.a_chk : &G.x_chk[cur];
         const bool sym_a = f.kind != kGram, sym_b = f.kind == kPoly, upd = f.kind == kUpdate;
         const int nsub = f.tw / TILE;
+        if (!WR && nsub > 1) {  // a 512-wide tile does not fit this ring's stages (host plan error)
+          record_status(p.status, kDevFault);
+          *abort_flag = 1;
+          break;
+        }
         const uint32_t bytes = 2 * (A_STAGE + nsub * B_STAGE);
         const int kblocks = (f.kind == kGram ? G.np : G.mp) / BK;
         const int arow = f.row0 + static_cast<int>(rank) * BM;
@@ -422,12 +442,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     const int e = warp - 2;                 // epilogue warp 0..7
     const int quad = warp & 3;              // TMEM lanes 32*quad .. 32*quad+31
     const int cbase = (e >> 2) * 128;       // this warp's first column within each half
-    uint8_t* otile = smem + EPI_OFFSET + e * 2 * EPI_OUT_BYTES;
+    uint8_t* wblock = smem + EPI_OFFSET + e * EPI_WARP_BYTES;  // this warp's own epilogue block
+    uint8_t* otile = wblock;
     const uint32_t otile_u32 = smem_u32(otile);
-    const uint8_t* abuf = smem + EPI_AUX_OFFSET + e * 2 * EPI_AUX_BYTES;  // this warp's two A chunks
+    const uint8_t* abuf = wblock + 2 * EPI_OUT_BYTES;  // this warp's two A chunks
     const uint32_t abuf_u32 = smem_u32(abuf);
     uint32_t naux = 0, nissued = 0;   // A chunks consumed / requested (their buffers alternate)
-    float* st32 = reinterpret_cast<float*>(smem + EPI_OFFSET + e * EPI_F32_BYTES);
+    float* st32 = reinterpret_cast<float*>(wblock);
     const int sub_r = lane >> 2, sub_c = (lane & 3) * 8;
     const int swz = (lane >> 1) & 3;  // 64-byte swizzle of this lane's staging row
     uint32_t uses[2] = {0u, 0u};
@@ -456,6 +477,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         ldw = tr ? G.m_real : G.n_real;
       }
       const bool wread = fw && p.w_decay != 0.0f && gr0 < G.m_real;
+      if (fw) {
+        // the fp32 staging overlays this warp's store tiles: no store of its may still read them
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
       auto woff = [&](int gc, int rr) -> size_t {
         return tr ? static_cast<size_t>(gc + rr) * ldw + gr0 + sub_c : static_cast<size_t>(gr0 + rr) * ldw + gc + sub_c;
       };
@@ -670,7 +696,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
 
 }  // namespace
 
-size_t fused_smem_bytes() { return SMEM_BYTES; }
+size_t fused_smem_bytes() { return FLayout<true>::SMEM_BYTES; }
 
 long long check_fused_tiles(const NsParams& p) {
   // Walk the tile list with the kernel's own decoding: every tile in range, every stored block of
@@ -746,25 +772,27 @@ long long check_fused_tiles(const NsParams& p) {
   return bad;
 }
 
-cudaError_t launch_ns_fused(const NsParams& p, int num_sms, cudaStream_t s) {
-  if (p.t_end <= p.t_begin) return cudaSuccess;
+namespace {
+
+template <bool WR>
+cudaError_t launch_fused_kind(const NsParams& p, int num_sms, cudaStream_t s) {
   static std::atomic<unsigned long long> attr_set{0};
   static std::atomic<int> max_clusters[64];
+  constexpr size_t smem = FLayout<WR>::SMEM_BYTES;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   const unsigned long long bit = 1ull << dev;
   if ((attr_set.load() & bit) == 0) {
-    e = cudaFuncSetAttribute(ns_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(SMEM_BYTES));
+    e = cudaFuncSetAttribute(ns_fused_kernel<WR>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     // Every pair must be resident at once (a tile may wait for a tile of any other pair): the
     // grid never exceeds the clusters of two that fit on the device together.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
     attr.val.clusterDim.x = 2;
@@ -773,15 +801,23 @@ cudaError_t launch_ns_fused(const NsParams& p, int num_sms, cudaStream_t s) {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, ns_fused_kernel, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, ns_fused_kernel<WR>, &cfg);
     if (e != cudaSuccess) return e;
     if (n < 1) return cudaErrorInvalidConfiguration;
     max_clusters[dev].store(n);
     attr_set.fetch_or(bit);
   }
   const int pairs = std::min({num_sms / 2, max_clusters[dev].load(), p.t_end - p.t_begin});
-  ns_fused_kernel<<<2 * pairs, kTcThreads, SMEM_BYTES, s>>>(p);
+  ns_fused_kernel<WR><<<2 * pairs, kTcThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_ns_fused(const NsParams& p, int num_sms, cudaStream_t s) {
+  if (p.t_end <= p.t_begin) return cudaSuccess;
+  const bool wide = p.upd_tw[0] > TILE || p.upd_tw[1] > TILE || p.sym_wide != 0;
+  return wide ? launch_fused_kind<true>(p, num_sms, s) : launch_fused_kind<false>(p, num_sms, s);
 }
 
 }  // namespace muon

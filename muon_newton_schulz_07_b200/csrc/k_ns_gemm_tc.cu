@@ -37,9 +37,10 @@
 // round-robin list of pair tiles):
 //   warp 0      TMA producer, one TMA per operand tile and k slice (a 64 x 128
 //               box for K-major tiles, a 4-D box of two 64-wide chunks for
-//               MN-major ones, 128-byte swizzle) into a ring of 4 stages of
-//               32 KB (3 of 48 KB for wide tiles); the even CTA's full barrier
-//               counts the bytes of both CTAs
+//               MN-major ones, 128-byte swizzle) into a ring of as many stages
+//               as shared memory holds (6 x 32 KB for Gram, 5 x 32 KB for Poly and
+//               the 256-wide Update, 4 x 48 KB for wide tiles); the even CTA's full
+//               barrier counts the bytes of both CTAs
 //   warp 1      TMEM allocation (512 columns: two 256-column accumulators, so
 //               the epilogue of one tile overlaps the main loop of the next, or
 //               one 512-column accumulator for wide tiles); in the even CTA,
@@ -67,32 +68,44 @@
 namespace muon {
 namespace {
 
-constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK, STAGES = kTcStages;
+constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK;
 constexpr int TILE = 256;                               // pair tile: 256 x 256
 constexpr uint32_t A_STAGE = BM * BK * 2;               // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t B_STAGE = (BN / 2) * BK * 2;         // 16 KB: this CTA's half of B
 constexpr uint32_t TMEM_COLS = 512;                     // 2 accumulators x 256 fp32 columns
-constexpr uint32_t BAR_BYTES = 256;
+constexpr uint32_t BAR_BYTES = 512;
 constexpr int F32_PITCH = 36;                            // staged fp32 row: 32 + 4 pad (144 B, 16-B aligned)
 constexpr int EPI_WARPS = kTcEpiWarps;
-// Shared memory: the stage ring (at most 144 KB: 4 x 32 KB for 256-wide tiles, 3 x 48 KB
-// for 512-wide ones), then per epilogue warp two 32 x 32 bf16 store tiles (2 KB each,
-// 64-byte swizzle), then per warp two 32 x 32 chunks of the polynomial's input A, loaded by
-// TMA two chunks ahead (same 64-byte swizzle).  The fp32 staging of the fused parameter write
-// reuses the start of the region (that launch makes no TMA stores and reads no A).
-constexpr uint32_t STAGE_REGION = 147456;
 constexpr uint32_t EPI_OUT_BYTES = 2048;
 constexpr uint32_t EPI_AUX_BYTES = 2048;
 constexpr uint32_t EPI_F32_BYTES = 32 * F32_PITCH * 4;
-constexpr uint32_t EPI_OFFSET = STAGE_REGION;            // 1024-byte aligned, as the swizzled tiles need
-constexpr uint32_t EPI_AUX_OFFSET = EPI_OFFSET + EPI_WARPS * 2 * EPI_OUT_BYTES;
-constexpr uint32_t BAR_OFFSET = EPI_AUX_OFFSET + EPI_WARPS * 2 * EPI_AUX_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + BAR_OFFSET + BAR_BYTES;
-// barriers: full[NST], empty[NST], accf[2], acce[2], the TMEM slot word, then two per epilogue
-// warp for its A chunks
-static_assert((2 * kTcStages + 5 + 2 * kTcEpiWarps) * 8 <= BAR_BYTES, "barriers must fit their region");
-static_assert(EPI_WARPS * EPI_F32_BYTES <= BAR_OFFSET - EPI_OFFSET, "fp32 staging must fit the epilogue region");
-static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+constexpr uint32_t SMEM_LIMIT = 232448;                 // 227 KB per CTA
+
+// Shared memory of one stage's kernel: the operand ring, then per epilogue warp two 32 x 32 bf16
+// store tiles (2 KB each, 64-byte swizzle), then (Poly) per warp two 32 x 32 chunks of the
+// polynomial's input A, loaded by TMA two chunks ahead (same swizzle); the fused parameter write
+// of the last Update stages fp32 chunks in the epilogue region instead.  The ring gets as many
+// stages as fit (at most 6): 6 x 32 KB for Gram, 5 x 32 KB for Poly and the 256-wide Update,
+// 4 x 48 KB for the 256 x 512 Update tiles, whose operands take longest to arrive.
+template <int KIND, bool WIDE>
+struct Layout {
+  static constexpr int NSUB = WIDE ? 2 : 1;
+  static constexpr uint32_t SB = A_STAGE + NSUB * B_STAGE;  // bytes of one stage in one CTA
+  static constexpr bool AUX = KIND == kPoly;
+  static constexpr uint32_t EPI = EPI_WARPS * 2 * EPI_OUT_BYTES + (AUX ? EPI_WARPS * 2 * EPI_AUX_BYTES : 0);
+  static constexpr uint32_t F32 = (KIND == kUpdate && !WIDE) ? EPI_WARPS * EPI_F32_BYTES : 0;
+  static constexpr uint32_t EPI_REGION = EPI > F32 ? EPI : F32;
+  static constexpr int FIT = static_cast<int>((SMEM_LIMIT - 1024 - BAR_BYTES - EPI_REGION) / SB);
+  static constexpr int NST = FIT < 6 ? FIT : 6;
+  static constexpr uint32_t EPI_OFFSET = NST * SB;          // 16 KB multiples: 1024-byte aligned
+  static constexpr uint32_t EPI_AUX_OFFSET = EPI_OFFSET + EPI_WARPS * 2 * EPI_OUT_BYTES;
+  static constexpr uint32_t BAR_OFFSET = EPI_OFFSET + EPI_REGION;
+  static constexpr size_t SMEM_BYTES = 1024 + BAR_OFFSET + BAR_BYTES;
+  static_assert(NST >= 3, "at least three operand stages");
+  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory per CTA");
+  // barriers: full[NST], empty[NST], accf[2], acce[2], the TMEM slot word, two per epilogue warp
+  static_assert((2 * NST + 5 + 2 * EPI_WARPS) * 8 <= BAR_BYTES, "barriers must fit their region");
+};
 
 struct Tile {
   int g, mat, row0, col0;
@@ -148,13 +161,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     ns_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   // WIDE (Update only): the pair tile is 256 x 512, two N = 256 MMAs per k step into one
   // 512-column accumulator, so every k slice of A feeds twice the columns.
-  constexpr int NSUB = WIDE ? 2 : 1;
+  using LY = Layout<KIND, WIDE>;
+  constexpr int NSUB = LY::NSUB;
   constexpr int TW = TILE * NSUB;                   // pair tile width
-  constexpr int NST = WIDE ? 3 : STAGES;
-  constexpr uint32_t SB = A_STAGE + NSUB * B_STAGE;  // bytes of one stage in one CTA
+  constexpr int NST = LY::NST;
+  constexpr uint32_t SB = LY::SB;                   // bytes of one stage in one CTA
+  constexpr uint32_t EPI_OFFSET = LY::EPI_OFFSET, EPI_AUX_OFFSET = LY::EPI_AUX_OFFSET, BAR_OFFSET = LY::BAR_OFFSET;
   constexpr int NACC = WIDE ? 1 : 2;                 // accumulators in TMEM
   static_assert(!WIDE || KIND == kUpdate, "wide tiles are for the Update only");
-  static_assert(NST * SB <= STAGE_REGION, "the stage ring must fit its region");
   static_assert(NACC * TW <= TMEM_COLS, "accumulators must fit TMEM");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -542,17 +556,17 @@ cudaError_t launch_kind(const TcParams& p, int grid, cudaStream_t s) {
   const unsigned long long bit = 1ull << (dev & 63);
   if ((attr_set.load() & bit) == 0) {
     e = cudaFuncSetAttribute(ns_gemm_tc_kernel<KIND, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(SMEM_BYTES));
+                             static_cast<int>(Layout<KIND, WIDE>::SMEM_BYTES));
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
-  ns_gemm_tc_kernel<KIND, WIDE><<<grid, kTcThreads, SMEM_BYTES, s>>>(p);
+  ns_gemm_tc_kernel<KIND, WIDE><<<grid, kTcThreads, Layout<KIND, WIDE>::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t tc_smem_bytes() { return SMEM_BYTES; }
+size_t tc_smem_bytes() { return Layout<kUpdate, true>::SMEM_BYTES; }
 
 cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;

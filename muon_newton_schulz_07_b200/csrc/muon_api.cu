@@ -303,16 +303,16 @@ bool fused_schedule(const muon_ctx* h, int k) {
 }
 
 // Tile tables of one momentum/norm launch (matrices b .. b+cnt-1), without the pointers and the
-// hyper-parameters: the persistent grid of num_sms * kEwCtasPerSm CTAs, CTA c taking tiles
-// c, c + G, ... of the launch's T tiles; a matrix gets one partial sum per warp of every CTA
-// that reaches it, min(ntiles, G) CTAs.
-void front_tables(const Plan& P, const std::vector<muon_shape_t>& shapes, int b, int cnt, int num_sms,
+// hyper-parameters: a persistent grid of G = min(ctas, tiles) CTAs, CTA c taking tiles c, c + G,
+// ... of the launch's T tiles; a matrix gets one partial sum per compute warp of every CTA that
+// reaches it, min(ntiles, G) CTAs.
+void front_tables(const Plan& P, const std::vector<muon_shape_t>& shapes, int b, int cnt, int ctas,
                   EwParams* prm) {
   std::memset(prm, 0, sizeof(*prm));
   prm->nmat = cnt;
   int total = 0;
   for (int j = 0; j < cnt; ++j) total += P.ew_ntiles[b + j];
-  const int grid = std::max(1, std::min({num_sms * kEwCtasPerSm, kEwMaxCtas, total}));
+  const int grid = std::max(1, std::min({ctas, kEwMaxCtas, total}));
   prm->total_tiles = total;
   prm->grid = grid;
   int tiles = 0, parts = 0;
@@ -354,14 +354,22 @@ cudaError_t enqueue_front(muon_ctx* h, const void* const* src, void* const* mom,
   EwParams& prm = h->ew;
   for (int b = 0; b < h->n; b += kEwMatsPerLaunch) {
     const int cnt = std::min(kEwMatsPerLaunch, h->n - b);
-    front_tables(P, h->shapes, b, cnt, h->num_sms, &prm);
+    // 16-byte aligned rows everywhere: the bulk-copy-fed kernel, one CTA per SM; else the
+    // register-fed one, kEwCtasPerSm per SM
+    int vec_ok = 1;
+    for (int j = 0; j < cnt; ++j) {
+      const int i = b + j;
+      const int vmul = (h->dtype == MUON_BF16) ? 8 : 4;
+      if (!aligned16(src[i]) || (mom && !aligned16(mom[i])) || (h->shapes[i].cols % vmul) != 0) vec_ok = 0;
+    }
+    front_tables(P, h->shapes, b, cnt, vec_ok ? h->num_sms : h->num_sms * kEwCtasPerSm, &prm);
     prm.beta = hp->beta;
     prm.eps = hp->eps;
     prm.nesterov = hp->nesterov ? 1 : 0;
     prm.partials = h->d_partials;
     prm.scal = h->d_scal;
     prm.norms = h->d_norms;
-    int vec_ok = 1;
+    prm.status = h->d_status;
     for (int j = 0; j < cnt; ++j) {
       const int i = b + j;
       const GroupPlan& gp = P.groups[P.mat_group[i]];
@@ -370,8 +378,6 @@ cudaError_t enqueue_front(muon_ctx* h, const void* const* src, void* const* mom,
       m.src = src[i];
       m.mom = mom ? mom[i] : nullptr;
       m.x = h->ws + gp.off_x[0] + static_cast<size_t>(P.mat_slot[i]) * gp.mp * gp.np * elem;
-      const int vmul = (h->dtype == MUON_BF16) ? 8 : 4;
-      if (!aligned16(m.src) || (m.mom && !aligned16(m.mom)) || (m.cols % vmul) != 0) vec_ok = 0;
     }
     prm.vec_ok = vec_ok;
     e = launch_momentum_norm(prm, io, xt, st);
@@ -393,7 +399,9 @@ void fused_tables(const Plan& P, int nslots, int k, bool fuse_write, NsParams* q
   for (const GroupPlan& gp : P.groups) wide = wide && gp.np % 512 == 0;
   q->upd_tw[0] = wide ? 512 : 256;
   q->upd_tw[1] = (wide && !fuse_write) ? 512 : 256;  // the Update that writes W keeps 256-wide tiles
-  q->sym_wide = 1;
+  // Gram and Poly keep one 256 x 256 block per tile: two blocks per tile (256 x 512, one
+  // accumulator, half of the epilogue exposed) measured 13 % (Gram) and 20 % (Poly) slower on d24
+  q->sym_wide = 0;
   for (int g = 0; g < ng; ++g) {
     const GroupPlan& gp = P.groups[g];
     NsGroup& G = q->g[g];
@@ -947,8 +955,10 @@ muon_status_t muon_check_plan(const muon_shape_t* shapes, int n, int ns_steps, i
     return MUON_ERR_INVALID_ARG;
   }
   for (int b = 0; b < n; b += kEwMatsPerLaunch) {
-    front_tables(P, sh, b, std::min(kEwMatsPerLaunch, n - b), num_sms, ew);
-    bad += check_front_tables(*ew);
+    for (int per_sm = 1; per_sm <= kEwCtasPerSm; ++per_sm) {  // both momentum kernels' grids
+      front_tables(P, sh, b, std::min(kEwMatsPerLaunch, n - b), num_sms * per_sm, ew);
+      bad += check_front_tables(*ew);
+    }
   }
   if (ns_steps >= 1 && P.groups.size() <= static_cast<size_t>(kTcMaxGroups)) {
     for (int fw = 0; fw < 2; ++fw) {

@@ -22,7 +22,8 @@ constexpr int kPad = 256;
 constexpr int kEwTileR = 64;
 constexpr int kEwTileC = 128;
 constexpr int kEwThreads = 256;
-constexpr int kEwCtasPerSm = 2;     // resident CTAs per SM of the persistent momentum/norm kernel
+constexpr int kEwCtasPerSm = 2;     // resident CTAs per SM of the register-fed momentum/norm kernel
+                                    // (the bulk-copy-fed one, for aligned launches, runs one per SM)
 constexpr int kEwMaxCtas = 4096;    // upper bound of its grid (sizes the per-CTA partial sums)
 constexpr int kEwMatsPerLaunch = 192;
 
@@ -58,6 +59,7 @@ struct EwParams {
   float* partials;         // per (matrix, CTA, warp) sums of squares
   float* scal;             // per matrix: {||U||_F, 1/(||U||_F + eps)}
   float* norms;            // ||U||_F per matrix, caller order
+  unsigned int* status;    // device status word (a bounded wait that ran out)
 };
 
 struct WrMat {
@@ -88,7 +90,6 @@ cudaError_t launch_param_write(const WrParams& p, Dtype io, Dtype xt, cudaStream
 constexpr int kTcBM = 128;
 constexpr int kTcBN = 256;
 constexpr int kTcBK = 64;
-constexpr int kTcStages = 4;       // 256-wide tiles: 4 x 32 KB; 512-wide tiles: 3 x 48 KB
 constexpr int kTcMaxGroups = 6;
 constexpr int kTcEpiWarps = 8;     // two per TMEM lane quadrant, each on half of the tile's columns
 constexpr int kTcThreads = 64 + 32 * kTcEpiWarps;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
