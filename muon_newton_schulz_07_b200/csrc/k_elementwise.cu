@@ -7,11 +7,10 @@
 //    影响 paragraph).  It reads G and M once, writes M1 in place and U (cast to
 //    the Newton-Schulz operand type) into the zero-padded, oriented workspace
 //    buffer X0.  Tall matrices are transposed through shared memory so X0 is
-//    always min x max.  The kernel is persistent (two CTAs per SM), CTA c
-//    taking every P-th tile from c on, with the next tile's loads in flight
-//    while it stores the current one.  The sum of squares goes warp -> one
-//    partial per (matrix, CTA, warp) in the workspace; norm_finish_kernel, the
-//    next launch, adds each matrix's partials in a fixed order, so the norm is
+//    always min x max.  One CTA per 64 x 128 tile, four CTAs per SM.  The sum
+//    of squares goes warp -> one partial per (CTA, warp)
+//    in the workspace; norm_finish_kernel, the next launch, adds each matrix's
+//    partials in a fixed order, so the norm is
 //    deterministic, and stores ||U|| and 1/(||U|| + eps) (0 when both are 0: a
 //    zero direction gives a zero update).  The normalisation itself is folded
 //    into the first Newton-Schulz products.
@@ -27,7 +26,6 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
-#include <atomic>
 #include <vector>
 
 #include "muon_device.cuh"
@@ -284,214 +282,37 @@ __device__ __forceinline__ float momentum_tile_store(const EwMat& mt, const EwPa
   return ss;
 }
 
-// The matrix of tile t, starting the search at matrix mi (t never lies before it).
-__device__ __forceinline__ int matrix_of_tile(const EwParams& p, int mi, int t) {
-  while (mi + 1 < p.nmat && t >= p.mat[mi + 1].tile_begin) ++mi;
-  return mi;
-}
-
-// This warp's part of matrix mt's sum of squares (the tiles this CTA took from mt) is complete:
-// one plain store into the warp's own slot.  CTA c reaches the tiles of mt whose index is
-// congruent to c modulo the grid, the first at offset r = (c - tile_begin) mod grid < nparts,
-// so slot (r, warp) is written by this warp alone.  No atomics and no fences: the sums are added
-// by norm_finish_kernel, the next launch on the stream.
-__device__ __forceinline__ void momentum_flush(const EwParams& p, const EwMat& mt, float ss) {
+// This warp's part of its matrix's sum of squares: one plain store into slot (CTA, warp), which
+// no other warp writes.  No atomics and no fences: the sums are added by norm_finish_kernel, the
+// next launch on the stream.
+__device__ __forceinline__ void momentum_flush(const EwParams& p, float ss) {
   ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) {
-    const int g = static_cast<int>(gridDim.x);
-    const int r = ((static_cast<int>(blockIdx.x) - mt.tile_begin) % g + g) % g;
-    p.partials[static_cast<size_t>(mt.part_begin + r) * (kEwThreads / 32) + (threadIdx.x >> 5)] = ss;
-  }
+  if ((threadIdx.x & 31) == 0)
+    p.partials[static_cast<size_t>(blockIdx.x) * (kEwThreads / 32) + (threadIdx.x >> 5)] = ss;
 }
 
-// Persistent: CTA c takes tiles c, c + P, c + 2P, ... of the launch (T tiles, P CTAs, matrices
-// back to back), so at any moment the CTAs work on neighbouring tiles (the same rows of the same
-// matrix, which keeps the DRAM pages they touch open) rather than on P distant streams.  For bf16
-// sources the loads of the next tile are issued before the current tile is computed and stored
-// (two register buffers), so every thread keeps eight 16-byte loads in flight while it works.
+// One CTA per 64 x 128 tile: CTA c works on tile c of the launch (matrix j owns CTAs part_begin ..
+// part_begin + nparts - 1, one per tile).  Each thread issues all eight of its 16-byte loads (G and
+// M of four 8-element chunks) before any arithmetic, and four CTAs share an SM, so 32 KB per CTA
+// (128 KB per SM) are in flight.  Short-lived CTAs rather than a persistent grid or several tiles
+// per CTA: the block scheduler starts a new tile the moment one ends, which kept DRAM busier than
+// every longer-lived form measured.
 template <typename T, typename XT>
-__global__ void __launch_bounds__(kEwThreads, kEwCtasPerSm) momentum_norm_kernel(const __grid_constant__ EwParams p) {
+__global__ void __launch_bounds__(kEwThreads, sizeof(T) == 2 ? kEwMinCtasPerSm : 2)
+    momentum_norm_kernel(const __grid_constant__ EwParams p) {
   constexpr int LD = kEwTileC + (sizeof(XT) == 2 ? 2 : 1);
   __shared__ XT stage[kEwTileR][LD];
-
-  const int step = static_cast<int>(gridDim.x);
-  const int t0 = static_cast<int>(blockIdx.x);
-  if (t0 >= p.total_tiles) return;
-  int lo = 0, hi = p.nmat - 1;  // matrix of t0
+  const int cta = static_cast<int>(blockIdx.x);
+  int lo = 0, hi = p.nmat - 1;  // the matrix whose CTA range holds this CTA
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (p.mat[mid].tile_begin <= t0) lo = mid; else hi = mid - 1;
+    if (p.mat[mid].part_begin <= cta) lo = mid; else hi = mid - 1;
   }
-  int mi = lo;          // matrix whose partial sum is being accumulated
-  float ss = 0.0f;
-  // bf16 sources: two register buffers (the next tile's loads in flight); fp32 sources hold
-  // twice the bytes per tile, so they keep one buffer and rely on the second resident CTA.
-  constexpr int NBUF = sizeof(T) == 2 ? 2 : 1;
-  MomentumChunks<T> buf[NBUF];
-  int mnext = mi;
-  if (NBUF == 2) momentum_tile_load<T>(p.mat[mi], p, t0 - p.mat[mi].tile_begin, buf[0]);
-#pragma unroll 1
-  for (int t = t0; t < p.total_tiles; t += NBUF * step) {
-#pragma unroll
-    for (int h = 0; h < NBUF; ++h) {
-      const int tt = t + h * step;
-      if (tt < p.total_tiles) {
-        int mcur;
-        if (NBUF == 2) {
-          mcur = mnext;
-          if (tt + step < p.total_tiles) {
-            mnext = matrix_of_tile(p, mcur, tt + step);
-            momentum_tile_load<T>(p.mat[mnext], p, tt + step - p.mat[mnext].tile_begin, buf[(h + 1) % NBUF]);
-          }
-        } else {
-          mcur = matrix_of_tile(p, mi, tt);
-          momentum_tile_load<T>(p.mat[mcur], p, tt - p.mat[mcur].tile_begin, buf[0]);
-        }
-        if (mcur != mi) {
-          momentum_flush(p, p.mat[mi], ss);
-          ss = 0.0f;
-          mi = mcur;
-        }
-        ss += momentum_tile_store<T, XT, LD>(p.mat[mi], p, tt - p.mat[mi].tile_begin, buf[h], stage);
-      }
-    }
-  }
-  momentum_flush(p, p.mat[mi], ss);
-}
-
-// ---------------------------------------------------------------- async-copy-fed variant
-// For launches whose sources are 16-byte aligned with rows a multiple of 8 elements (vec_ok): one
-// CTA of 256 threads per SM, each thread streaming its own 16-byte pieces of G and M for the next
-// kAsyncStages - 1 tiles into shared memory with cp.async (no registers held for data in flight),
-// then computing a tile from its own pieces.  Five tiles (160 KB for bf16) are in flight per SM.
-template <typename T> struct AsyncGeometry {
-  static constexpr int STAGE = 2 * kEwTileR * kEwTileC * static_cast<int>(sizeof(T));  // G and M of one tile
-  static constexpr int STAGES = sizeof(T) == 2 ? 5 : 3;
-};
-
-template <typename T, typename XT>
-size_t async_smem_bytes() {
-  constexpr int LD = kEwTileC + (sizeof(XT) == 2 ? 2 : 1);
-  return static_cast<size_t>(AsyncGeometry<T>::STAGES) * AsyncGeometry<T>::STAGE +
-         static_cast<size_t>(kEwTileR) * LD * sizeof(XT);
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// The 16-byte pieces of tile t (matrix mt) this thread works on, G and M, into its slots of one
-// stage: piece (q, which) of thread i sits at ((which * 4 + q) * kEwThreads + i) pieces from the
-// stage's start, so neighbouring threads touch neighbouring 16 bytes.  Pieces outside the matrix
-// are not copied (momentum_chunk gives them U = 0 without reading).
-template <typename T>
-__device__ __forceinline__ void momentum_tile_async(const EwMat& mt, int t, uint32_t stage) {
-  constexpr int PIECE = 16;
-  constexpr int PER8 = static_cast<int>(sizeof(T)) * 8 / PIECE;  // 16-byte pieces per 8 elements
-  const int xr0 = (t / mt.tiles_c) * kEwTileR;
-  const int xc0 = (t % mt.tiles_c) * kEwTileC;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = threadIdx.x + q * kEwThreads;
-    const int row = mt.trans ? xc0 + (c >> 3) : xr0 + (c >> 4);
-    const int col = mt.trans ? xr0 + (c & 7) * 8 : xc0 + (c & 15) * 8;
-    if (row < mt.rows && col + 8 <= mt.cols) {
-      const size_t base = static_cast<size_t>(row) * mt.cols + col;
-#pragma unroll
-      for (int h = 0; h < PER8; ++h) {
-        const uint32_t off = static_cast<uint32_t>(((0 * 4 + q) * PER8 + h) * kEwThreads + threadIdx.x) * PIECE;
-        cp_async16(stage + off, static_cast<const T*>(mt.src) + base + h * (8 / PER8));
-        if (mt.mom != nullptr) {
-          const uint32_t offm = static_cast<uint32_t>(((1 * 4 + q) * PER8 + h) * kEwThreads + threadIdx.x) * PIECE;
-          cp_async16(stage + offm, static_cast<const T*>(mt.mom) + base + h * (8 / PER8));
-        }
-      }
-    }
-  }
-}
-
-// The pieces of tile t this thread copied into stage `st`, as MomentumChunks.
-template <typename T>
-__device__ __forceinline__ void momentum_tile_from_async(const EwMat& mt, int t, const uint8_t* st,
-                                                         MomentumChunks<T>& c) {
-  constexpr int PIECE = 16;
-  constexpr int PER8 = static_cast<int>(sizeof(T)) * 8 / PIECE;
-  const int xr0 = (t / mt.tiles_c) * kEwTileR;
-  const int xc0 = (t % mt.tiles_c) * kEwTileC;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int cc = threadIdx.x + q * kEwThreads;
-    const int row = mt.trans ? xc0 + (cc >> 3) : xr0 + (cc >> 4);
-    const int col = mt.trans ? xr0 + (cc & 7) * 8 : xc0 + (cc & 15) * 8;
-    c.vec[q] = row < mt.rows && col + 8 <= mt.cols;
-    if (c.vec[q]) {
-#pragma unroll
-      for (int h = 0; h < PER8; ++h) {
-        reinterpret_cast<uint4*>(&c.g[q])[h] =
-            *reinterpret_cast<const uint4*>(st + (((0 * 4 + q) * PER8 + h) * kEwThreads + threadIdx.x) * PIECE);
-        if (mt.mom != nullptr)
-          reinterpret_cast<uint4*>(&c.m[q])[h] =
-              *reinterpret_cast<const uint4*>(st + (((1 * 4 + q) * PER8 + h) * kEwThreads + threadIdx.x) * PIECE);
-      }
-    }
-  }
-}
-
-template <typename T, typename XT>
-__global__ void __launch_bounds__(kEwThreads, 1) momentum_norm_async_kernel(const __grid_constant__ EwParams p) {
-  constexpr int LD = kEwTileC + (sizeof(XT) == 2 ? 2 : 1);
-  constexpr int NS = AsyncGeometry<T>::STAGES;
-  constexpr int SB = AsyncGeometry<T>::STAGE;
-  extern __shared__ __align__(16) uint8_t smem_async[];
-  XT(*stage)[LD] = reinterpret_cast<XT(*)[LD]>(smem_async + NS * SB);
-  const uint32_t ring = smem_u32(smem_async);
-  const int step = static_cast<int>(gridDim.x);
-  const int t0 = static_cast<int>(blockIdx.x);
-  if (t0 >= p.total_tiles) return;
-  int lo = 0, hi = p.nmat - 1;  // matrix of t0
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.mat[mid].tile_begin <= t0) lo = mid; else hi = mid - 1;
-  }
-  // prologue: the first NS - 1 tiles of this CTA on their way (one copy group per tile)
-  int mload = lo;
-#pragma unroll 1
-  for (int k = 0; k < NS - 1; ++k) {
-    const int t = t0 + k * step;
-    if (t < p.total_tiles) {
-      mload = matrix_of_tile(p, mload, t);
-      momentum_tile_async<T>(p.mat[mload], t - p.mat[mload].tile_begin, ring + k * SB);
-    }
-    cp_async_commit();
-  }
-  int mi = lo, macc = lo, j = 0;
-  float ss = 0.0f;
-#pragma unroll 1
-  for (int t = t0; t < p.total_tiles; t += step, ++j) {
-    // the tile NS - 1 ahead into the slot the previous iteration has finished reading
-    const int tn = t + (NS - 1) * step;
-    if (tn < p.total_tiles) {
-      mload = matrix_of_tile(p, mload, tn);
-      momentum_tile_async<T>(p.mat[mload], tn - p.mat[mload].tile_begin, ring + ((j + NS - 1) % NS) * SB);
-    }
-    cp_async_commit();
-    cp_async_wait<NS - 1>();   // this thread's pieces of tile t have landed
-    mi = matrix_of_tile(p, mi, t);
-    const EwMat& mt = p.mat[mi];
-    MomentumChunks<T> ch;
-    momentum_tile_from_async<T>(mt, t - mt.tile_begin, smem_async + (j % NS) * SB, ch);
-    if (mi != macc) {
-      momentum_flush(p, p.mat[macc], ss);
-      ss = 0.0f;
-      macc = mi;
-    }
-    ss += momentum_tile_store<T, XT, LD>(mt, p, t - mt.tile_begin, ch, stage);
-  }
-  cp_async_wait<0>();
-  momentum_flush(p, p.mat[macc], ss);
+  const EwMat& mt = p.mat[lo];
+  const int t = cta - mt.part_begin;
+  MomentumChunks<T> ch;
+  momentum_tile_load<T>(mt, p, t, ch);
+  momentum_flush(p, momentum_tile_store<T, XT, LD>(mt, p, t, ch, stage));
 }
 
 // The norms of one momentum/norm launch's matrices: CTA j adds matrix j's per-warp partial sums
@@ -620,26 +441,8 @@ __global__ void __launch_bounds__(kEwThreads, 3) param_write_kernel(const __grid
 
 template <typename T, typename XT>
 cudaError_t launch_mn(const EwParams& p, cudaStream_t s) {
-  cudaError_t e;
-  if (p.vec_ok) {
-    // async-copy-fed: one CTA per SM (the tables were built for that grid)
-    static std::atomic<unsigned long long> attr_set{0};
-    int dev = 0;
-    e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    const size_t smem = async_smem_bytes<T, XT>();
-    if ((attr_set.load() & bit) == 0) {
-      e = cudaFuncSetAttribute(momentum_norm_async_kernel<T, XT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      attr_set.fetch_or(bit);
-    }
-    momentum_norm_async_kernel<T, XT><<<p.grid, kEwThreads, smem, s>>>(p);
-  } else {
-    momentum_norm_kernel<T, XT><<<p.grid, kEwThreads, 0, s>>>(p);
-  }
-  e = cudaGetLastError();
+  momentum_norm_kernel<T, XT><<<p.grid, kEwThreads, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   norm_finish_kernel<<<p.nmat, kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
@@ -653,39 +456,20 @@ cudaError_t launch_wr(const WrParams& p, cudaStream_t s) {
 }  // namespace
 
 long long check_front_tables(const EwParams& p) {
-  // Replay the persistent kernel's walk on the host: the matrices' tile ranges back to back, and
-  // each matrix's partial sums written once per CTA that reaches it (the CTA's first tile of the
-  // matrix at offset r < nparts) into slots [part_begin, part_begin + nparts), no slot twice.
+  // The matrices' tile ranges back to back, one CTA (one partial-sum slot per warp) per tile, so
+  // each matrix's CTA range is its tile range; the grid is the launch's tile count.
   long long bad = 0;
-  if (p.nmat < 1 || p.nmat > kEwMatsPerLaunch || p.grid < 1 || p.grid > kEwMaxCtas || p.grid > p.total_tiles)
-    return 1;
-  int tiles = 0, parts = 0;
+  if (p.nmat < 1 || p.nmat > kEwMatsPerLaunch) return 1;
+  long long tiles = 0;
   for (int j = 0; j < p.nmat; ++j) {
     const EwMat& m = p.mat[j];
-    if (m.tile_begin != tiles || m.ntiles < 1 || m.part_begin != parts || m.nparts != std::min(m.ntiles, p.grid) ||
-        m.tiles_c * kEwTileC != m.np || m.ntiles * kEwTileR * kEwTileC != m.mp * m.np)
+    if (m.tile_begin != tiles || m.ntiles < 1 || m.part_begin != m.tile_begin || m.nparts != m.ntiles ||
+        m.tiles_c * kEwTileC != m.np ||
+        static_cast<long long>(m.ntiles) * kEwTileR * kEwTileC != static_cast<long long>(m.mp) * m.np)
       ++bad;
     tiles += m.ntiles;
-    parts += m.nparts;
   }
-  if (tiles != p.total_tiles) ++bad;
-  std::vector<int> written(static_cast<size_t>(parts > 0 ? parts : 1), 0);
-  for (int c = 0; c < p.grid; ++c) {
-    int mi = -1;
-    for (int t = c; t < p.total_tiles; t += p.grid) {
-      int mt = 0;
-      while (mt + 1 < p.nmat && t >= p.mat[mt + 1].tile_begin) ++mt;
-      if (mt != mi) {  // this CTA's flush of matrix mt
-        const EwMat& m = p.mat[mt];
-        const int r = ((c - m.tile_begin) % p.grid + p.grid) % p.grid;
-        if (r != t - m.tile_begin || r >= m.nparts) ++bad;
-        else ++written[m.part_begin + r];
-        mi = mt;
-      }
-    }
-  }
-  for (int i = 0; i < parts; ++i)
-    if (written[i] != 1) ++bad;
+  if (tiles != p.total_tiles || tiles != p.grid || p.grid < 1) ++bad;
   return bad;
 }
 

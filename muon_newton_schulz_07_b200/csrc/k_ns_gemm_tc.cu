@@ -421,6 +421,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       const float cdiag = (KIND == kPoly && gr < G.m_real) ? p.c_diag : 0.0f;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * TW);
       const uint32_t acce_leader = map_to_rank(acce_bar(acc), 0);
+      if constexpr (WIDE) {
+        // (never the Update that writes the parameters: the host keeps that one 256 wide)
+        // One accumulator, so the MMA issuer waits for it: read this warp's whole part (32 rows
+        // x 256 columns) into registers as the bf16 values it will store, hand the accumulator
+        // back, and only then stage and store the chunks.  (Chunk by chunk, the stores of the
+        // first seven chunks would sit between the issuer and its next tile.)
+        uint32_t pk[NW][16];
+#pragma unroll
+        for (int c = 0; c < NW; ++c) {
+          float v[32];
+          tmem_ld_32cols(taddr + (ch0 + c) * 32, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(s * p.c_acc * v[2 * i], s * p.c_acc * v[2 * i + 1]);
+            pk[c][i] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acce_leader);
+#pragma unroll
+        for (int c = 0; c < NW; ++c) {
+          const uint32_t ob = (c & 1) * EPI_OUT_BYTES;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(otile + ob + lane * 64 + ((q ^ swz) << 4)) =
+                make_uint4(pk[c][4 * q], pk[c][4 * q + 1], pk[c][4 * q + 2], pk[c][4 * q + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&G.tm_out, otile_u32 + ob, ti.col0 + (ch0 + c) * 32, gr0, ti.mat);
+            bulk_commit();
+          }
+        }
+      } else {
 #pragma unroll 1
       for (int c = 0; c < NW; ++c) {
         const int ch = ch0 + c;
@@ -519,6 +556,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         }
       }
       if (aux) naux += NW;  // (an early exit leaves naux behind nissued; see the drain below)
+      }
       if (++acc == NACC) {
         acc = 0;
         acc_phase ^= 1u;
@@ -570,6 +608,7 @@ size_t tc_smem_bytes() { return Layout<kUpdate, true>::SMEM_BYTES; }
 
 cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;
+  if (p.wide && (p.kind != kUpdate || p.fuse_write)) return cudaErrorInvalidValue;  // 256-wide only
   // one CTA pair per TPC, at most one pair per tile
   const int grid = 2 * std::min(num_sms / 2, p.total_tiles);
   if (p.kind == kGram) return launch_kind<kGram, false>(p, grid, s);

@@ -124,10 +124,10 @@ void make_plan(const muon_shape_t* shapes, int n, muon_mode_t mode, Plan* P) {
     const GroupPlan& gp = P->groups[P->mat_group[i]];
     P->ew_ntiles[i] = (gp.mp / kEwTileR) * (gp.np / kEwTileC);
   }
-  // One partial sum per (matrix, CTA, warp) of the persistent momentum/norm kernel, min(ntiles,
-  // grid) CTAs per matrix; launches in sequence reuse the buffer, so the whole set bounds it.
+  // One partial sum per (CTA, warp) of the momentum/norm kernel, one CTA per tile; launches in
+  // sequence reuse the buffer, so the whole set bounds it.
   size_t parts = 0;
-  for (int i = 0; i < n; ++i) parts += static_cast<size_t>(std::min(P->ew_ntiles[i], kEwMaxCtas)) * (kEwThreads / 32);
+  for (int i = 0; i < n; ++i) parts += static_cast<size_t>(P->ew_ntiles[i]) * (kEwThreads / 32);
   size_t off = 0;
   P->off_status = off;
   off = align_up(off + 64, 1024);
@@ -303,18 +303,10 @@ bool fused_schedule(const muon_ctx* h, int k) {
 }
 
 // Tile tables of one momentum/norm launch (matrices b .. b+cnt-1), without the pointers and the
-// hyper-parameters: a persistent grid of G = min(ctas, tiles) CTAs, CTA c taking tiles c, c + G,
-// ... of the launch's T tiles; a matrix gets one partial sum per compute warp of every CTA that
-// reaches it, min(ntiles, G) CTAs.
-void front_tables(const Plan& P, const std::vector<muon_shape_t>& shapes, int b, int cnt, int ctas,
-                  EwParams* prm) {
+// hyper-parameters: one CTA per tile, the matrices' tiles back to back.
+void front_tables(const Plan& P, const std::vector<muon_shape_t>& shapes, int b, int cnt, EwParams* prm) {
   std::memset(prm, 0, sizeof(*prm));
   prm->nmat = cnt;
-  int total = 0;
-  for (int j = 0; j < cnt; ++j) total += P.ew_ntiles[b + j];
-  const int grid = std::max(1, std::min({ctas, kEwMaxCtas, total}));
-  prm->total_tiles = total;
-  prm->grid = grid;
   int tiles = 0, parts = 0;
   for (int j = 0; j < cnt; ++j) {
     const int i = b + j;
@@ -330,11 +322,13 @@ void front_tables(const Plan& P, const std::vector<muon_shape_t>& shapes, int b,
     m.ntiles = P.ew_ntiles[i];
     m.scal_idx = P.scal_idx[i];
     m.caller_idx = i;
-    m.nparts = std::min(m.ntiles, grid);
+    m.nparts = m.ntiles;
     m.part_begin = parts;
     parts += m.nparts;
     tiles += m.ntiles;
   }
+  prm->total_tiles = tiles;
+  prm->grid = parts;
 }
 
 // The elementwise front end (momentum + norm + orientation) over all matrices.
@@ -354,15 +348,14 @@ cudaError_t enqueue_front(muon_ctx* h, const void* const* src, void* const* mom,
   EwParams& prm = h->ew;
   for (int b = 0; b < h->n; b += kEwMatsPerLaunch) {
     const int cnt = std::min(kEwMatsPerLaunch, h->n - b);
-    // 16-byte aligned rows everywhere: the bulk-copy-fed kernel, one CTA per SM; else the
-    // register-fed one, kEwCtasPerSm per SM
+    // 16-byte aligned rows everywhere: vector accesses (else element by element)
     int vec_ok = 1;
     for (int j = 0; j < cnt; ++j) {
       const int i = b + j;
       const int vmul = (h->dtype == MUON_BF16) ? 8 : 4;
       if (!aligned16(src[i]) || (mom && !aligned16(mom[i])) || (h->shapes[i].cols % vmul) != 0) vec_ok = 0;
     }
-    front_tables(P, h->shapes, b, cnt, vec_ok ? h->num_sms : h->num_sms * kEwCtasPerSm, &prm);
+    front_tables(P, h->shapes, b, cnt, &prm);
     prm.beta = hp->beta;
     prm.eps = hp->eps;
     prm.nesterov = hp->nesterov ? 1 : 0;
@@ -941,7 +934,7 @@ muon_status_t muon_get_plan(muon_handle_t h, int ns_steps, int* n_groups, int* l
 
 muon_status_t muon_check_plan(const muon_shape_t* shapes, int n, int ns_steps, int num_sms, int64_t* problems) {
   if (problems == nullptr || !shapes_ok(shapes, n) || ns_steps < 0 || ns_steps > 64 || num_sms < 2 ||
-      num_sms > kEwMaxCtas)
+      num_sms > 4096)
     return MUON_ERR_INVALID_ARG;
   Plan P;
   make_plan(shapes, n, MUON_MODE_FAST, &P);
@@ -955,10 +948,8 @@ muon_status_t muon_check_plan(const muon_shape_t* shapes, int n, int ns_steps, i
     return MUON_ERR_INVALID_ARG;
   }
   for (int b = 0; b < n; b += kEwMatsPerLaunch) {
-    for (int per_sm = 1; per_sm <= kEwCtasPerSm; ++per_sm) {  // both momentum kernels' grids
-      front_tables(P, sh, b, std::min(kEwMatsPerLaunch, n - b), num_sms * per_sm, ew);
-      bad += check_front_tables(*ew);
-    }
+    front_tables(P, sh, b, std::min(kEwMatsPerLaunch, n - b), ew);
+    bad += check_front_tables(*ew);
   }
   if (ns_steps >= 1 && P.groups.size() <= static_cast<size_t>(kTcMaxGroups)) {
     for (int fw = 0; fw < 2; ++fw) {

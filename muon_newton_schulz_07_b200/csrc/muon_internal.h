@@ -22,9 +22,7 @@ constexpr int kPad = 256;
 constexpr int kEwTileR = 64;
 constexpr int kEwTileC = 128;
 constexpr int kEwThreads = 256;
-constexpr int kEwCtasPerSm = 2;     // resident CTAs per SM of the register-fed momentum/norm kernel
-                                    // (the bulk-copy-fed one, for aligned launches, runs one per SM)
-constexpr int kEwMaxCtas = 4096;    // upper bound of its grid (sizes the per-CTA partial sums)
+constexpr int kEwMinCtasPerSm = 4;  // resident momentum/norm CTAs per SM the register budget allows (bf16 sources)
 constexpr int kEwMatsPerLaunch = 192;
 
 enum Dtype : int { kBF16 = 0, kF32 = 1 };
@@ -41,22 +39,21 @@ struct EwMat {
   int ntiles;        // X tiles of the padded matrix (mp/64 * np/128)
   int scal_idx;      // slot of this matrix in the scalar / counter tables
   int caller_idx;    // position in the caller's matrix list
-  int part_begin;    // first partial-sum slot of this matrix (a slot holds one sum per warp)
-  int nparts;        // CTAs that reach this matrix: min(ntiles, grid)
+  int part_begin;    // first CTA of this matrix in the launch (= tile_begin: one CTA per tile)
+  int nparts;        // CTAs of this matrix, each with one partial-sum slot per warp (= ntiles)
 };
 
-// The momentum/norm kernel is persistent: CTA c of a grid of P takes tiles c, c + P, c + 2P, ...
-// of the launch's T tiles (matrices back to back).
+// The momentum/norm launch: one CTA per tile, matrix j's CTAs part_begin .. part_begin + nparts - 1.
 struct EwParams {
   EwMat mat[kEwMatsPerLaunch];
   int nmat;
   int total_tiles;
-  int grid;
+  int grid;                // CTAs of the launch: the sum of the matrices' nparts
   float beta;
   float eps;
   int nesterov;
   int vec_ok;              // every row of every matrix starts 16-byte aligned
-  float* partials;         // per (matrix, CTA, warp) sums of squares
+  float* partials;         // per (CTA, warp) sums of squares
   float* scal;             // per matrix: {||U||_F, 1/(||U||_F + eps)}
   float* norms;            // ||U||_F per matrix, caller order
   unsigned int* status;    // device status word (a bounded wait that ran out)
