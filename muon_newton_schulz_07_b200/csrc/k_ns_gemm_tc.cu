@@ -33,20 +33,23 @@
 // L2 per multiply-add, at the price of one 512-column accumulator (the epilogue
 // of a tile no longer overlaps the main loop of the next).
 //
-// Roles in each CTA (320 threads, one CTA per SM, persistent over a static
-// round-robin list of pair tiles):
+// Roles in each CTA (320 threads, 576 for Poly; one CTA per SM,
+// persistent over a static round-robin list of pair tiles):
 //   warp 0      TMA producer, one TMA per operand tile and k slice (a 64 x 128
 //               box for K-major tiles, a 4-D box of two 64-wide chunks for
 //               MN-major ones, 128-byte swizzle) into a ring of as many stages
-//               as shared memory holds (6 x 32 KB for Gram, 5 x 32 KB for Poly and
-//               the 256-wide Update, 4 x 48 KB for wide tiles); the even CTA's full
+//               as shared memory holds (6 x 32 KB for Gram, 5 x 32 KB for Poly
+//               and the 256-wide Update, 4 x 48 KB for 512-wide tiles); the even
+//               CTA's full
 //               barrier counts the bytes of both CTAs
 //   warp 1      TMEM allocation (512 columns: two 256-column accumulators, so
 //               the epilogue of one tile overlaps the main loop of the next, or
 //               one 512-column accumulator for wide tiles); in the even CTA,
 //               lane 0 issues the MMAs
-//   warps 2..9  epilogue, two warps per TMEM lane quadrant, each on half of the
-//               tile's columns: tcgen05.ld 32 columns at a time, the fp32
+//   warps 2..    epilogue: 8 warps, two per TMEM lane quadrant, each on half of the
+//               tile's columns; Poly 16, four per quadrant, each on a quarter (its
+//               epilogue reads A as well and its k loop is short): tcgen05.ld 32
+//               columns at a time, the fp32
 //               combination (Poly: c A A + b A + a I), bf16 pack into a
 //               64B-swizzled 32 x 32 staging tile, one TMA store per chunk
 //               (upper blocks only for Gram/Poly).  In the last Update the
@@ -75,36 +78,42 @@ constexpr uint32_t B_STAGE = (BN / 2) * BK * 2;         // 16 KB: this CTA's hal
 constexpr uint32_t TMEM_COLS = 512;                     // 2 accumulators x 256 fp32 columns
 constexpr uint32_t BAR_BYTES = 512;
 constexpr int F32_PITCH = 36;                            // staged fp32 row: 32 + 4 pad (144 B, 16-B aligned)
-constexpr int EPI_WARPS = kTcEpiWarps;
 constexpr uint32_t EPI_OUT_BYTES = 2048;
 constexpr uint32_t EPI_AUX_BYTES = 2048;
 constexpr uint32_t EPI_F32_BYTES = 32 * F32_PITCH * 4;
 constexpr uint32_t SMEM_LIMIT = 232448;                 // 227 KB per CTA
 
 // Shared memory of one stage's kernel: the operand ring, then per epilogue warp two 32 x 32 bf16
-// store tiles (2 KB each, 64-byte swizzle), then (Poly) per warp two 32 x 32 chunks of the
-// polynomial's input A, loaded by TMA two chunks ahead (same swizzle); the fused parameter write
-// of the last Update stages fp32 chunks in the epilogue region instead.  The ring gets as many
-// stages as fit (at most 6): 6 x 32 KB for Gram, 5 x 32 KB for Poly and the 256-wide Update,
-// 4 x 48 KB for the 256 x 512 Update tiles, whose operands take longest to arrive.
+// store tiles (2 KB each, 64-byte swizzle).  Poly's epilogue loads each 32 x 32 chunk of its
+// input A by TMA into the store tile that chunk's result will leave from (same swizzle); the
+// fused parameter write of the last Update stages fp32 chunks in the epilogue region instead.
+// The ring gets as many stages as fit (at most 6): 6 x 32 KB for Gram, 5 x 32 KB for Poly and
+// the 256-wide Update, 4 x 48 KB for the 256 x 512 Update tiles (ring depths from 4 to 6
+// measured the same).
 template <int KIND, bool WIDE>
 struct Layout {
+  // Epilogue warps: 8 (two per TMEM lane quadrant), 16 for Poly (four per quadrant, each on a
+  // quarter of the tile's columns), whose epilogue does the most work per multiply-add.
+  static constexpr int EW = KIND == kPoly ? 2 * kTcEpiWarps : kTcEpiWarps;
+  static constexpr int THREADS = 64 + 32 * EW;
   static constexpr int NSUB = WIDE ? 2 : 1;
   static constexpr uint32_t SB = A_STAGE + NSUB * B_STAGE;  // bytes of one stage in one CTA
   static constexpr bool AUX = KIND == kPoly;
-  static constexpr uint32_t EPI = EPI_WARPS * 2 * EPI_OUT_BYTES + (AUX ? EPI_WARPS * 2 * EPI_AUX_BYTES : 0);
-  static constexpr uint32_t F32 = (KIND == kUpdate && !WIDE) ? EPI_WARPS * EPI_F32_BYTES : 0;
+  // Poly loads each chunk of its input A into the store tile the chunk's result leaves from.
+  static constexpr uint32_t EPI = EW * 2 * EPI_OUT_BYTES;
+  static constexpr uint32_t F32 = (KIND == kUpdate && !WIDE) ? EW * EPI_F32_BYTES : 0;
   static constexpr uint32_t EPI_REGION = EPI > F32 ? EPI : F32;
   static constexpr int FIT = static_cast<int>((SMEM_LIMIT - 1024 - BAR_BYTES - EPI_REGION) / SB);
   static constexpr int NST = FIT < 6 ? FIT : 6;
   static constexpr uint32_t EPI_OFFSET = NST * SB;          // 16 KB multiples: 1024-byte aligned
-  static constexpr uint32_t EPI_AUX_OFFSET = EPI_OFFSET + EPI_WARPS * 2 * EPI_OUT_BYTES;
+  static constexpr uint32_t EPI_AUX_OFFSET = EPI_OFFSET;   // shares the store tiles
+  static_assert(EPI_AUX_BYTES == EPI_OUT_BYTES, "an A chunk and a result chunk share a tile");
   static constexpr uint32_t BAR_OFFSET = EPI_OFFSET + EPI_REGION;
   static constexpr size_t SMEM_BYTES = 1024 + BAR_OFFSET + BAR_BYTES;
   static_assert(NST >= 3, "at least three operand stages");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory per CTA");
   // barriers: full[NST], empty[NST], accf[2], acce[2], the TMEM slot word, two per epilogue warp
-  static_assert((2 * NST + 5 + 2 * EPI_WARPS) * 8 <= BAR_BYTES, "barriers must fit their region");
+  static_assert((2 * NST + 5 + 2 * EW) * 8 <= BAR_BYTES, "barriers must fit their region");
 };
 
 struct Tile {
@@ -157,11 +166,12 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 }
 
 template <int KIND, bool WIDE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Layout<KIND, WIDE>::THREADS, 1)
     ns_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   // WIDE (Update only): the pair tile is 256 x 512, two N = 256 MMAs per k step into one
   // 512-column accumulator, so every k slice of A feeds twice the columns.
   using LY = Layout<KIND, WIDE>;
+  constexpr int EPI_WARPS = LY::EW;
   constexpr int NSUB = LY::NSUB;
   constexpr int TW = TILE * NSUB;                   // pair tile width
   constexpr int NST = LY::NST;
@@ -340,19 +350,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    // Eight warps, two per TMEM lane quadrant: each owns 32 rows of the CTA's 128 and half
-    // of the tile's columns, which it walks in 32 x 32 chunks.  A finished chunk is packed
+    // EPI_WARPS warps, EPI_WARPS / 4 per TMEM lane quadrant: each owns 32 rows of the CTA's 128
+    // and its share of the tile's columns, which it walks in 32 x 32 chunks.  A finished chunk is packed
     // to bf16 into one of the warp's two 32 x 32 staging tiles (64-byte rows, 64-byte
     // swizzle, so the row-per-lane writes are free of bank conflicts) and written to global
     // memory by one TMA store.  The fused parameter write goes through an fp32 staging tile
     // and plain stores instead, since W is the caller's memory.
-    const int e = warp - 2;                 // epilogue warp 0..7
+    const int e = warp - 2;                 // epilogue warp 0 .. EPI_WARPS-1
     const int quad = warp & 3;              // TMEM lanes 32*quad .. 32*quad+31
-    constexpr int NW = TW / 64;             // chunks per warp and tile
+    constexpr int NW = TW / (8 * EPI_WARPS);  // chunks per warp and tile (32 columns each)
+    static_assert(KIND != kPoly || NW % 2 == 0, "A chunk naux + c and result chunk c share tile c & 1");
     const int ch0 = (e >> 2) * NW;          // this warp's first chunk
     uint8_t* otile = smem + EPI_OFFSET + e * 2 * EPI_OUT_BYTES;
     const uint32_t otile_u32 = smem_u32(otile);
-    const uint8_t* abuf = smem + EPI_AUX_OFFSET + e * 2 * EPI_AUX_BYTES;  // this warp's two A chunks
+    const uint8_t* abuf = smem + EPI_AUX_OFFSET + e * 2 * EPI_AUX_BYTES;  // = otile: A in, B' out
     const uint32_t abuf_u32 = smem_u32(abuf);
     float* st32 = reinterpret_cast<float*>(smem + EPI_OFFSET + e * EPI_F32_BYTES);
     const int sub_r = lane >> 2, sub_c = (lane & 3) * 8;
@@ -369,7 +380,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       const int gr0 = ti.row0 + static_cast<int>(rank) * BM + quad * 32;  // first row of this warp
       const int gr = gr0 + lane;
       // Fused parameter write (last Update): the caller's matrix of this tile.
-      const bool fw = p.fuse_write != 0;
+      const bool fw = KIND == kUpdate && !WIDE && p.fuse_write != 0;
       __nv_bfloat16* W = nullptr;
       float cw = 0.0f;
       bool tr = false;
@@ -398,6 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
                     ti.mat);
       };
       if (aux && lane == 0) {
+        bulk_wait_read<0>();  // the previous tile's last stores have left both tiles
         aux_issue(0);
         if (NW > 1) aux_issue(1);
       }
@@ -525,12 +537,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[8 * q + i] = s * fmaf(p.c_acc, v[8 * q + i], p.c_aux * a8[i]);
           }
-          // every lane has used its row: the buffer may take the chunk two ahead
-          __syncwarp();
-          if (lane == 0 && c + 2 < NW) {
-            fence_async_smem();
-            aux_issue(c + 2);
-          }
+          __syncwarp();  // every lane has read its row of A: the tile takes the result next
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = s * p.c_acc * v[i];
@@ -553,6 +560,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
           tma_store_3d(&G.tm_out, otile_u32 + ob, gc0, gr0, ti.mat);
           bulk_commit();
+          if (aux && c + 2 < NW) {
+            // the tile takes the chunk of A two ahead once this store has read it
+            bulk_wait_read<0>();
+            aux_issue(c + 2);
+          }
         }
       }
       if (aux) naux += NW;  // (an early exit leaves naux behind nissued; see the drain below)
@@ -598,7 +610,7 @@ cudaError_t launch_kind(const TcParams& p, int grid, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
-  ns_gemm_tc_kernel<KIND, WIDE><<<grid, kTcThreads, Layout<KIND, WIDE>::SMEM_BYTES, s>>>(p);
+  ns_gemm_tc_kernel<KIND, WIDE><<<grid, Layout<KIND, WIDE>::THREADS, Layout<KIND, WIDE>::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
