@@ -54,8 +54,9 @@
 //               64B-swizzled 32 x 32 staging tile, one TMA store per chunk
 //               (upper blocks only for Gram/Poly).  In the last Update the
 //               epilogue writes the parameters directly:
-//               W = (1 - lr wd) W - lr sqrt(max(1, r/c)) X_k from the unrounded
-//               fp32 X_k, transposed back for tall matrices.
+//               W = (1 - lr wd) W - lr sqrt(max(1, r/c)) X_k, transposed back for
+//               tall matrices, from the unrounded fp32 X_k (256-wide tiles) or from
+//               X_k rounded to bf16 as the separate write kernel reads it (512-wide).
 // Operand B of Update is X itself in its row-major layout, i.e. MN-major, and so
 // is every transposed block of A or B'; the other operands are K-major.  The
 // instruction descriptor's major bits are set per k slice.  All waits are
@@ -98,7 +99,6 @@ struct Layout {
   static constexpr int THREADS = 64 + 32 * EW;
   static constexpr int NSUB = WIDE ? 2 : 1;
   static constexpr uint32_t SB = A_STAGE + NSUB * B_STAGE;  // bytes of one stage in one CTA
-  static constexpr bool AUX = KIND == kPoly;
   // Poly loads each chunk of its input A into the store tile the chunk's result leaves from.
   static constexpr uint32_t EPI = EW * 2 * EPI_OUT_BYTES;
   static constexpr uint32_t F32 = (KIND == kUpdate && !WIDE) ? EW * EPI_F32_BYTES : 0;
@@ -380,7 +380,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Layout<KIND, WIDE>::
       const int gr0 = ti.row0 + static_cast<int>(rank) * BM + quad * 32;  // first row of this warp
       const int gr = gr0 + lane;
       // Fused parameter write (last Update): the caller's matrix of this tile.
-      const bool fw = KIND == kUpdate && !WIDE && p.fuse_write != 0;
+      const bool fw = KIND == kUpdate && p.fuse_write != 0;
       __nv_bfloat16* W = nullptr;
       float cw = 0.0f;
       bool tr = false;
@@ -421,7 +421,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Layout<KIND, WIDE>::
           for (int q = 0; q < 4; ++q) dst[q] = __ldcs(reinterpret_cast<const uint4*>(W + woff(gc, q * 8 + sub_r)));
         }
       };
-      const bool has_pre = wread;
+      const bool has_pre = wread && !WIDE;  // (the wide path loads W after reading the accumulator)
       if (has_pre) pre_load(ch0, pf);
       if (!mbar_wait_bounded(accf_bar(acc), acc_phase, tmo, abort_flag, p.status)) break;
       tc_fence_after();
@@ -434,11 +434,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Layout<KIND, WIDE>::
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * TW);
       const uint32_t acce_leader = map_to_rank(acce_bar(acc), 0);
       if constexpr (WIDE) {
-        // (never the Update that writes the parameters: the host keeps that one 256 wide)
         // One accumulator, so the MMA issuer waits for it: read this warp's whole part (32 rows
-        // x 256 columns) into registers as the bf16 values it will store, hand the accumulator
-        // back, and only then stage and store the chunks.  (Chunk by chunk, the stores of the
-        // first seven chunks would sit between the issuer and its next tile.)
+        // x 256 columns) into registers as bf16 (the X_k the workspace would hold), hand the
+        // accumulator back, and only then stage and store the chunks.  (Chunk by chunk, the
+        // stores of the first seven chunks would sit between the issuer and its next tile.)
+        // When the launch writes the parameters, each chunk goes through a padded row-major
+        // staging tile (read column-wise for tall parameters) into W = w_decay W + coef X_k, the
+        // arithmetic of param_write_kernel on the same bf16 X_k.
         uint32_t pk[NW][16];
 #pragma unroll
         for (int c = 0; c < NW; ++c) {
@@ -453,6 +455,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Layout<KIND, WIDE>::
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(acce_leader);
+        if (fw) {
+          constexpr int PITCH = 80;  // bytes per staged row: 32 bf16 + 16 (16-byte aligned, conflict-free)
+          static_assert(32 * PITCH <= 2 * EPI_OUT_BYTES, "the staging tile fits the warp's two store tiles");
+          uint8_t* stg = otile;
+#pragma unroll
+          for (int c = 0; c < NW; ++c) {
+            const int gc0 = ti.col0 + (ch0 + c) * 32;
+            if (gr0 < G.m_real && gc0 < G.n_real) {  // the padding has no parameters
+              uint4 w4[4];
+              if (wread) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  w4[q] = __ldcs(reinterpret_cast<const uint4*>(W + woff(gc0, q * 8 + sub_r)));
+              }
+              __syncwarp();  // the previous chunk's staged rows have been read
+              // row r of the staged tile = row r of this chunk of X_k
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4*>(stg + lane * PITCH + q * 16) =
+                    make_uint4(pk[c][4 * q], pk[c][4 * q + 1], pk[c][4 * q + 2], pk[c][4 * q + 3]);
+              __syncwarp();
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int rr = q * 8 + sub_r;
+                float x8[8], r8[8];
+                if (!tr) {
+                  unpack8(*reinterpret_cast<const uint4*>(stg + rr * PITCH + sub_c * 2), x8);
+                } else {
+                  // W row gc0 + rr, columns gr0 + sub_c .. +7: column rr of staged rows sub_c ..
+#pragma unroll
+                  for (int j = 0; j < 8; ++j)
+                    x8[j] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(stg + (sub_c + j) * PITCH + rr * 2));
+                }
+                if (wread) {
+                  float w8[8];
+                  unpack8(w4[q], w8);
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) r8[i] = fmaf(p.w_decay, w8[i], cw * x8[i]);
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) r8[i] = cw * x8[i];
+                }
+                __stcs(reinterpret_cast<uint4*>(W + woff(gc0, rr)), pack8(r8));
+              }
+            }
+          }
+        } else {
 #pragma unroll
         for (int c = 0; c < NW; ++c) {
           const uint32_t ob = (c & 1) * EPI_OUT_BYTES;
@@ -468,6 +517,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Layout<KIND, WIDE>::
             tma_store_3d(&G.tm_out, otile_u32 + ob, ti.col0 + (ch0 + c) * 32, gr0, ti.mat);
             bulk_commit();
           }
+        }
         }
       } else {
 #pragma unroll 1
@@ -620,7 +670,7 @@ size_t tc_smem_bytes() { return Layout<kUpdate, true>::SMEM_BYTES; }
 
 cudaError_t launch_tc_gemm(const TcParams& p, int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;
-  if (p.wide && (p.kind != kUpdate || p.fuse_write)) return cudaErrorInvalidValue;  // 256-wide only
+  if (p.wide && p.kind != kUpdate) return cudaErrorInvalidValue;  // 256-wide only
   // one CTA pair per TPC, at most one pair per tile
   const int grid = 2 * std::min(num_sms / 2, p.total_tiles);
   if (p.kind == kGram) return launch_kind<kGram, false>(p, grid, s);

@@ -1,8 +1,9 @@
 """GPU parity of the step's less common branches against the float64 oracle, element by element.
 
 * nesterov = False (U = M1), and beta other than 0.95;
-* weight decay != 0 on both parameter-write paths: fused into the last Update (bf16 parameters
-  whose dimensions are all multiples of 32) and param_write_kernel (fp32 parameters, and bf16 sets
+* weight decay != 0 on every parameter-write path: fused into the last Update (bf16 parameters
+  whose dimensions are all multiples of 32; 256-wide tiles, and 512-wide tiles for long k loops)
+  and param_write_kernel (fp32 parameters, and bf16 sets
   with a dimension that is not a multiple of 32).  lr * wd = 0.002 is the usual setting, but with
   bf16 parameters 0.002 |W| is below half a bf16 spacing of W, so a decay factor of 0.9 is checked
   as well: there a wrong factor cannot hide in the rounding;
@@ -34,6 +35,9 @@ TOL_O = {"fast": 2e-2, "fp32_ref": 1e-4}
 # (name, shapes, storage dtype, mode, which write path the handle must take)
 SETS = [
     ("fused_d24_shapes", [(1536, 1536), (1536, 6144), (6144, 1536)], torch.bfloat16, "fast", "fused"),
+    # long k loops (m = 2048): the writing Update runs 256 x 512 tiles, its parameter write
+    # staged from registers after the accumulator is handed back (wide and tall parameters)
+    ("fused_wide_write", [(2048, 2048), (4096, 2048), (2048, 4096)], torch.bfloat16, "fast", "fused"),
     ("write_kernel_ragged_bf16", [(200, 328), (328, 200), (512, 768)], torch.bfloat16, "fast", "kernel"),
     ("write_kernel_fp32", [(256, 512), (512, 256), (320, 320)], torch.float32, "fast", "kernel"),
     ("fp32_reference_mode", [(257, 129), (130, 130)], torch.float32, "fp32_ref", "kernel"),
