@@ -423,6 +423,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Layout<KIND, WIDE>::
       };
       const bool has_pre = wread && !WIDE;  // (the wide path loads W after reading the accumulator)
       if (has_pre) pre_load(ch0, pf);
+      if (WIDE && wread && (lane & 3) == 0) {
+        // The wide path writes W only after the accumulator is back: pull this warp's rows of
+        // W for the whole tile into L2 now, while the tile's MMAs run (no registers held).
+#pragma unroll 1
+        for (int c = 0; c < NW; ++c) {
+          const int gc = ti.col0 + (ch0 + c) * 32;
+          if (gc < G.n_real) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) prefetch_l2(W + woff(gc, q * 8 + sub_r));
+          }
+        }
+      }
       if (!mbar_wait_bounded(accf_bar(acc), acc_phase, tmo, abort_flag, p.status)) break;
       tc_fence_after();
       float s = 1.0f;

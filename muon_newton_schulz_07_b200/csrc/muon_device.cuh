@@ -126,6 +126,10 @@ __device__ __forceinline__ bool wait_counter_bounded(const unsigned int* ctr, un
 
 // ---------------------------------------------------------------- TMA
 
+// Bring the line holding `p` into L2 (no register, no completion to wait for).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
