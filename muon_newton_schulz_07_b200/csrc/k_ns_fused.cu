@@ -568,16 +568,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           }
           if (fw) {
             // Last Update: write the parameters instead of X_k (no chunk straddles the padding:
-            // real dimensions are multiples of 32).
+            // real dimensions are multiples of 32), from X_k as its bf16 store would hold it, so
+            // the write is exactly param_write_kernel's on the stored X_k.
             if (gr0 < G.m_real && gc0 < G.n_real) {
               if (!tr) {
 #pragma unroll
                 for (int i = 0; i < 32; i += 4)
                   *reinterpret_cast<float4*>(st32 + lane * F32_PITCH + i) =
-                      make_float4(s * v[i], s * v[i + 1], s * v[i + 2], s * v[i + 3]);
+                      make_float4(bf16_round(s * v[i]), bf16_round(s * v[i + 1]), bf16_round(s * v[i + 2]),
+                                bf16_round(s * v[i + 3]));
               } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) st32[i * F32_PITCH + lane] = s * v[i];
+                for (int i = 0; i < 32; ++i) st32[i * F32_PITCH + lane] = bf16_round(s * v[i]);
               }
               __syncwarp();
 #pragma unroll

@@ -55,8 +55,8 @@
 //               (upper blocks only for Gram/Poly).  In the last Update the
 //               epilogue writes the parameters directly:
 //               W = (1 - lr wd) W - lr sqrt(max(1, r/c)) X_k, transposed back for
-//               tall matrices, from the unrounded fp32 X_k (256-wide tiles) or from
-//               X_k rounded to bf16 as the separate write kernel reads it (512-wide).
+//               tall matrices, from X_k rounded to bf16 exactly as the separate
+//               write kernel reads it from the workspace.
 // Operand B of Update is X itself in its row-major layout, i.e. MN-major, and so
 // is every transposed block of A or B'; the other operands are K-major.  The
 // instruction descriptor's major bits are set per k slice.  All waits are
@@ -551,15 +551,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Layout<KIND, WIDE>::
           // Last Update: write the parameters instead of X_k.  Chunks in the zero padding
           // of the workspace have no parameters (real dimensions are multiples of 32).
           if (gr0 < G.m_real && gc0 < G.n_real) {
-            // stage s * acc in fp32 (row-major, or transposed for tall parameters)
+            // stage X_k = s * acc as its bf16 store would hold it (so the write is exactly
+            // param_write_kernel's on the stored X_k), row-major or transposed for tall parameters
             if (!tr) {
 #pragma unroll
               for (int i = 0; i < 32; i += 4)
                 *reinterpret_cast<float4*>(st32 + lane * F32_PITCH + i) =
-                    make_float4(s * v[i], s * v[i + 1], s * v[i + 2], s * v[i + 3]);
+                    make_float4(bf16_round(s * v[i]), bf16_round(s * v[i + 1]), bf16_round(s * v[i + 2]),
+                                bf16_round(s * v[i + 3]));
             } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) st32[i * F32_PITCH + lane] = s * v[i];
+              for (int i = 0; i < 32; ++i) st32[i * F32_PITCH + lane] = bf16_round(s * v[i]);
             }
             __syncwarp();
 #pragma unroll

@@ -126,6 +126,9 @@ __device__ __forceinline__ bool wait_counter_bounded(const unsigned int* ctr, un
 
 // ---------------------------------------------------------------- TMA
 
+// x rounded to bf16 (nearest even) and back: the value a bf16 store of x would hold.
+__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
 // Bring the line holding `p` into L2 (no register, no completion to wait for).
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));

@@ -67,7 +67,7 @@ def assert_m1_elementwise(M1_gpu, M1_ref, M0, G0, dtype, what="M1"):
 
 
 def assert_w1_elementwise(W1_gpu, W1_ref, Wz_gpu, Wz_ref, W0, dtype, what="W1"):
-    """W1 = round(d W + c O) with O the kernel's own (unrounded) direction.  A step from the same
+    """W1 = round(d W + c O) with O the kernel's own direction as it applies it.  A step from the same
     momentum with W = 0 stores Wz = round(c O), so per element |c O - Wz_ref| <= |Wz - Wz_ref| +
     half a spacing of Wz, where Wz_ref is the oracle's step from W = 0.  W1 may then differ from
     the oracle's W1 by that direction error plus its own rounding (half a spacing)."""

@@ -137,3 +137,32 @@ def test_zero_direction_only_decays(shapes, dtype, mode, path, eps):
     err = np.abs(to_f64(W[0]) - decayed)
     assert np.all(err <= 0.5 * storage_ulp(decayed, dtype) + 2.0 ** -21 * np.abs(W0))
     op.close()
+
+
+@pytest.mark.parametrize("shapes", [[(1536, 1536), (1536, 6144), (6144, 1536)],
+                                    [(2048, 2048), (4096, 2048), (2048, 4096)]],
+                         ids=["256_wide_tiles", "512_wide_tiles"])
+def test_fused_write_equals_write_kernel(shapes):
+    # Every write path computes W1 = (1 - lr wd) W - lr s X_k from the same bf16 X_k with the same
+    # fused multiply-add, so the write fused into the last Update (16-byte aligned parameters) and
+    # param_write_kernel (the same parameters one element off a 16-byte boundary) agree bit for bit.
+    hp = dict(lr=0.05, beta=0.9, weight_decay=2.0, nesterov=True)
+    W, G, M = inputs(shapes, torch.bfloat16, 91)
+    Wk = []
+    for w in W:
+        base = torch.empty(w.numel() + 1, dtype=w.dtype, device=w.device)
+        view = base[1:].view(w.shape)
+        view.copy_(w)
+        assert view.data_ptr() % 16 != 0
+        Wk.append(view)
+    Mk = [m.clone() for m in M]
+    op = MuonStep(shapes, dtype=torch.bfloat16)
+    op(W, G, M, ns_steps=5, **hp)
+    op(Wk, G, Mk, ns_steps=5, **hp)
+    torch.cuda.synchronize()
+    assert op.status() == B.MUON_OK
+    for a, b in zip(M, Mk):
+        assert torch.equal(a, b)
+    bad = [i for i, (a, b) in enumerate(zip(W, Wk)) if not torch.equal(a, b)]
+    assert not bad, bad
+    op.close()
