@@ -32,7 +32,9 @@
  * iterations, then the parameter write.  In MUON_MODE_FAST the iterations run
  * as three tensor-core launches each (Gram, polynomial, update) over every
  * matrix of the handle, with the parameter write fused into the last update
- * for bf16 sets whose dimensions are multiples of 32.  When every matrix fits
+ * for bf16 sets whose dimensions are multiples of 32 and whose parameters are
+ * 16-byte aligned (the fused write and the separate write kernel compute the
+ * same W, bit for bit, from X_k rounded to bf16).  When every matrix fits
  * one 256 x 256 tile (max(rows, cols) <= 256, at most six distinct shapes),
  * all k iterations run in one launch instead (MUON_KERNEL_NS_SMALL).
  * Results are the same function of the inputs on either path, within the
