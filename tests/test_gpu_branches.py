@@ -66,7 +66,10 @@ def expected_launches(op, path, k):
         return 2 + 3 * k * op.n_groups + 1
     if path == "small":
         return 2 + 1 + 1   # every iteration in one launch, then the write kernel
-    return 2 + 3 * k + (0 if path == "fused" else 1)
+    # the default schedule runs every iteration in one launch when every shape group is at most
+    # 768 wide, else one launch per stage
+    single = all(-(-min(s) // 256) * 256 <= 768 for s in op.shapes)
+    return 2 + (1 if single else 3 * k) + (0 if path == "fused" else 1)
 
 
 def check_step(shapes, dtype, mode, path, hp, seed, k=5, eps=1e-7, zero=()):

@@ -97,8 +97,17 @@ def test_small_set_step_matches_oracle():
 
 
 def test_larger_sets_keep_the_general_path():
-    op = MuonStep([(256, 256), (256, 512)])
-    X = [torch.randn(s, device="cuda").to(torch.bfloat16) for s in op.shapes]
+    # a set that does not fit one 256 x 256 tile per matrix leaves the small-matrix kernel: one
+    # launch per stage when staged, one launch for every iteration by default (its groups are at
+    # most 768 wide)
+    staged = MuonStep([(256, 256), (256, 512)], schedule="staged")
+    X = [torch.randn(s, device="cuda").to(torch.bfloat16) for s in staged.shapes]
     Os = [torch.empty_like(x) for x in X]
-    kinds = launches_and_kinds(op, lambda: op.orthogonalize(X, Os, ns_steps=2))
+    kinds = launches_and_kinds(staged, lambda: staged.orthogonalize(X, Os, ns_steps=2))
     assert "ns_small" not in kinds and kinds.get("gram") == 2, kinds
+    auto = MuonStep([(256, 256), (256, 512)])
+    Oa = [torch.empty_like(x) for x in X]
+    kinds = launches_and_kinds(auto, lambda: auto.orthogonalize(X, Oa, ns_steps=2))
+    assert "ns_small" not in kinds and "gram" not in kinds and kinds.get("ns_fused") == 1, kinds
+    for a, b in zip(Oa, Os):
+        assert torch.equal(a, b)
