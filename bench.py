@@ -472,6 +472,15 @@ EXTRA_LEGS = {
 }
 
 
+def ns_schedule_taken(kern):
+    """How the Newton-Schulz iterations ran, from the kernels the trace saw."""
+    if "ns_small" in kern:
+        return "small-matrix kernel: every iteration of a matrix on chip, one launch"
+    if "ns_fused" in kern:
+        return "single launch: every stage of every iteration"
+    return "staged: one launch per stage"
+
+
 def run_extra_leg(leg, warmup, dev, local_rank, peaks, peak_src, schedule="auto", cache=None, graph=False):
     """One further workload leg; `cache` keeps the last workload's inputs for the next leg."""
     import torch
@@ -508,7 +517,7 @@ def run_extra_leg(leg, warmup, dev, local_rank, peaks, peak_src, schedule="auto"
                                            wl.name)
     ms = ms_total / steps
     out = {"workload": wl.name, "ns_steps": k, "matrices": len(shapes), "params": I.param_count(wl),
-           "steps": steps, "warmup": warmup, "ms_per_step": ms, "value": 1000.0 / ms, "unit": UNIT,
+           "schedule": schedule, "ns_schedule": ns_schedule_taken(kern), "steps": steps, "warmup": warmup, "ms_per_step": ms, "value": 1000.0 / ms, "unit": UNIT,
            "roofline": roof, "ns": ns, "kernels": kern, "targets": targets,
            "gpu_launches": op.launches_per_step(k) * steps, "clocks": clk,
            "l2": "flushed before every timed step" if flushed else "inputs larger than L2, no flush",
@@ -691,7 +700,7 @@ def run_muon(args, rank, world, local_rank):
             "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "matrices": n, "params": I.param_count(wl), "ns_steps": k,
-                       "groups": op.n_groups, "schedule": args.schedule,
+                       "groups": op.n_groups, "schedule": args.schedule, "ns_schedule": ns_schedule_taken(kern),
                        "parallelism": (f"sharded by matrix over {world} ranks + all-gather of W (NCCL)" if sharded
                                        else f"replica x{world} (one parameter set per GPU)"),
                        "l2": ("inputs larger than L2 (W, G, M: %.2f GB per GPU), no flush" % (in_bytes / 1e9)

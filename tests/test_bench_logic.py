@@ -100,3 +100,10 @@ def test_kernel_table_uses_the_burst_peak_for_the_headline():
     assert "write" not in kern
     assert set(targets) == {"ns_frac_of_burst_peak", "momentum_norm_frac_of_hbm"}
     assert targets["momentum_norm_frac_of_hbm"]["met"] == (kern["momentum_norm"]["frac_of_hbm"] >= 0.80)
+
+
+def test_ns_schedule_is_read_from_the_traced_kernels():
+    import bench
+    assert bench.ns_schedule_taken({"momentum_norm": {}, "ns_fused": {}}).startswith("single launch")
+    assert bench.ns_schedule_taken({"momentum_norm": {}, "ns_small": {}}).startswith("small-matrix")
+    assert bench.ns_schedule_taken({"momentum_norm": {}, "gram": {}, "poly": {}, "update": {}}).startswith("staged")
