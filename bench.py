@@ -134,7 +134,7 @@ class ClockSampler:
             os.close(fd)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -464,11 +464,14 @@ def timed_steps(step_fn, G_sets, steps, warmup, op, dev, stream, local_rank, syn
 
 
 # Further workloads timed after the headline one (one GPU only), each its own block of the line.
+# (workload, Newton-Schulz steps, timed steps): every timed region at least about half a second,
+# long enough for the GPU to reach the clock its power cap holds (a 70 ms region of the GPT-2-small
+# set ran before the cap had pulled the clock down) and for the clock sampler to see it.
 EXTRA_LEGS = {
-    "l38b": ("l38b", 5, 10),      # (workload, Newton-Schulz steps, timed steps)
-    "stress_k5": ("stress", 5, 20),
-    "stress_k10": ("stress", 10, 10),
-    "gpt2s": ("gpt2s", 5, 50),
+    "l38b": ("l38b", 5, 10),
+    "stress_k5": ("stress", 5, 30),
+    "stress_k10": ("stress", 10, 15),
+    "gpt2s": ("gpt2s", 5, 400),
 }
 
 
