@@ -35,6 +35,9 @@ SETS = {
     "ragged": [(200, 328), (328, 200), (520, 1000), (300, 300)],
     # six groups, the most one launch takes
     "six_groups": [(256, 512), (512, 768), (768, 1024), (1024, 256), (300, 1300), (512, 512)],
+    # long k loops (m = 2048): the staged schedule's last Update writes O from 512-wide tiles, the
+    # single launch from 256-wide ones; both from the same bf16 X_k
+    "long_k": [(2048, 2048), (4096, 2048), (2048, 4096)],
 }
 
 
